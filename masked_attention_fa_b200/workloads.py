@@ -1,0 +1,163 @@
+"""Seeded synthetic workloads (shapes, arguments and random inputs).
+
+This module only draws inputs and states shapes and call arguments; it holds
+none of the attention arithmetic, so both the CUDA path and the fp64 oracle
+can take their inputs from it without sharing any of the method.
+
+Input recipe (every workload): a CPU ``torch.Generator`` seeded with the
+workload's seed draws, in this order, the varlen lengths (TND workloads
+only), then q, k and v as float32 N(0, 1) which are rounded to bfloat16.
+The scale is 1/sqrt(D).
+
+The five named workloads follow the shapes of the Ascend "sparseMode参数说明"
+page's scenarios (band, leftUpCausal, right-down band, varlen
+rightDownCausal, prefix) at sizes of long-context inference.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import torch
+
+LAYOUTS = ("BNSD", "BSND", "TND")
+
+
+@dataclasses.dataclass
+class Workload:
+    name: str
+    layout: str
+    B: int
+    N: int
+    Sq: int
+    Skv: int
+    D: int
+    sparse_mode: int
+    pre_tokens: int = 0
+    next_tokens: int = 0
+    seed: int = 0
+    mask_kind: Optional[str] = None      # "SS", "B1SS", "BNSS" or None
+    prefix: Optional[list] = None        # modes 5/6, one entry per batch
+    actual_seq_qlen: Optional[list] = None   # TND cumulative ends (no leading 0)
+    actual_seq_kvlen: Optional[list] = None
+    scale: Optional[float] = None
+
+    def __post_init__(self):
+        if self.scale is None:
+            self.scale = 1.0 / math.sqrt(self.D)
+
+    def q_shape(self):
+        if self.layout == "BNSD":
+            return (self.B, self.N, self.Sq, self.D)
+        if self.layout == "BSND":
+            return (self.B, self.Sq, self.N, self.D)
+        return (self.Sq, self.N, self.D)
+
+    def kv_shape(self):
+        if self.layout == "BNSD":
+            return (self.B, self.N, self.Skv, self.D)
+        if self.layout == "BSND":
+            return (self.B, self.Skv, self.N, self.D)
+        return (self.Skv, self.N, self.D)
+
+    def lse_shape(self):
+        if self.layout == "TND":
+            return (self.N, self.Sq)
+        return (self.B, self.N, self.Sq)
+
+    def mask_shape(self):
+        if self.mask_kind == "SS":
+            return (self.Sq, self.Skv)
+        if self.mask_kind == "B1SS":
+            return (self.B, 1, self.Sq, self.Skv)
+        if self.mask_kind == "BNSS":
+            return (self.B, self.N, self.Sq, self.Skv)
+        return None
+
+    def seq_lens(self):
+        """[(Sq_b, Skv_b)] per sequence."""
+        if self.layout != "TND":
+            return [(self.Sq, self.Skv)] * self.B
+        out, pq, pk = [], 0, 0
+        for cq, ck in zip(self.actual_seq_qlen, self.actual_seq_kvlen):
+            out.append((cq - pq, ck - pk))
+            pq, pk = cq, ck
+        return out
+
+
+def varlen_lengths(gen: torch.Generator, nseq: int, q_lo: int, q_hi: int, extra_hi: int):
+    """Draw varlen lengths: Sq_b uniform in [q_lo, q_hi], Skv_b = Sq_b + uniform[0, extra_hi].
+
+    Returns the cumulative end-offset arrays (no leading 0).
+    """
+    sq = torch.randint(q_lo, q_hi + 1, (nseq,), generator=gen)
+    extra = torch.randint(0, extra_hi + 1, (nseq,), generator=gen)
+    skv = sq + extra
+    return torch.cumsum(sq, 0).tolist(), torch.cumsum(skv, 0).tolist()
+
+
+def lower_triangular_mask(S: int) -> torch.Tensor:
+    """The S x S lower-triangular attenMask the band page asks for in the causal
+    case (1 = masked, i.e. the strictly upper triangle)."""
+    return torch.triu(torch.ones(S, S, dtype=torch.uint8), diagonal=1)
+
+
+def named_workloads() -> dict:
+    """The five long-context scenarios, by name."""
+    g4 = torch.Generator("cpu").manual_seed(4)
+    cu_q, cu_kv = varlen_lengths(g4, 16, 512, 4096, 1024)
+    return {
+        # band from the top-left via preTokens/nextTokens, with the
+        # lower-triangular attenMask the page asks for (causal via band)
+        "band_causal_256": Workload("band_causal_256", "BNSD", 1, 2, 256, 256, 64, 0,
+                                    pre_tokens=256, next_tokens=0, seed=1, mask_kind="SS"),
+        "leftup_causal_4k": Workload("leftup_causal_4k", "BNSD", 2, 16, 4096, 4096, 128, 2,
+                                     seed=2),
+        "rightdown_band_2k_8k": Workload("rightdown_band_2k_8k", "BSND", 1, 32, 2048, 8192, 128,
+                                         4, pre_tokens=1024, next_tokens=0, seed=3),
+        "varlen_rightdown_16seq": Workload("varlen_rightdown_16seq", "TND", 16, 32, cu_q[-1],
+                                           cu_kv[-1], 128, 3, seed=4, actual_seq_qlen=cu_q,
+                                           actual_seq_kvlen=cu_kv),
+        "prefix_8k": Workload("prefix_8k", "BNSD", 4, 16, 8192, 8192, 128, 5, seed=5,
+                              prefix=[512, 1024, 2048, 4096]),
+    }
+
+
+def make_inputs(w: Workload, device="cpu"):
+    """Draw q, k, v (bf16) and the mask for workload w with its seed.
+
+    Returns a dict with q, k, v (on `device`) and mask (uint8 on `device`, or
+    None). TND lengths are part of the workload itself.
+    """
+    g = torch.Generator("cpu").manual_seed(w.seed)
+    if w.layout == "TND" and w.name == "varlen_rightdown_16seq":
+        # the lengths were drawn first from the same seed; redraw to advance
+        varlen_lengths(g, 16, 512, 4096, 1024)
+    q = torch.randn(w.q_shape(), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    k = torch.randn(w.kv_shape(), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    v = torch.randn(w.kv_shape(), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    mask = None
+    if w.mask_kind is not None:
+        if w.name == "band_causal_256":
+            mask = lower_triangular_mask(w.Sq)
+        else:
+            mask = (torch.rand(w.mask_shape(), generator=g) < 0.3).to(torch.uint8)
+    out = {"q": q.to(device), "k": k.to(device), "v": v.to(device),
+           "mask": None if mask is None else mask.to(device)}
+    return out
+
+
+def random_inputs(layout, B, N, Sq, Skv, D, seed, mask_kind=None, mask_density=0.3,
+                  device="cpu"):
+    """q, k, v (bf16 N(0,1)) and an optional Bernoulli(mask_density) mask."""
+    w = Workload("random", layout, B, N, Sq, Skv, D, 0, seed=seed, mask_kind=mask_kind)
+    g = torch.Generator("cpu").manual_seed(seed)
+    q = torch.randn(w.q_shape(), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    k = torch.randn(w.kv_shape(), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    v = torch.randn(w.kv_shape(), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    mask = None
+    if mask_kind is not None:
+        mask = (torch.rand(w.mask_shape(), generator=g) < mask_density).to(torch.uint8)
+    return {"q": q.to(device), "k": k.to(device), "v": v.to(device),
+            "mask": None if mask is None else mask.to(device)}

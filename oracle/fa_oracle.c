@@ -1,0 +1,412 @@
+/*
+ * Oracle for the masked attention forward: plain, slow, fp64 CPU code.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is the independent checker that the
+ * CUDA path is compared against. Nothing in the product path includes, links
+ * or calls it; it shares no header, helper or constant with the CUDA library.
+ * Only the test suite, the smoke check and the benchmark's CPU-baseline leg
+ * load it.
+ *
+ * What it computes, and where each step comes from:
+ *   - Visibility of key j to query i (the "Masked QK^T" geometry) for every
+ *     sparseMode 0..8, decided element by element from the prose of the
+ *     Ascend CANN page "sparseMode参数说明" (sections sparseMode=0 .. =8) and
+ *     the attenMask rule on the same page (a True mask entry hides that QK^T
+ *     position).
+ *   - The attention itself as its plain definition: S = scale * Q K^T,
+ *     softmax over the visible keys of each row, O = P V, and the per-row
+ *     natural log-sum-exp. A row with no visible key gives O = 0, lse = -inf.
+ *   - The tiled online-softmax recurrence (running max m_i, running sum l_i,
+ *     normalised output) of the "FlashAttention tiling & online softmax"
+ *     exercise page (section "Mục tiêu kiến thức"), used only to pin the
+ *     recurrence against the unfused softmax.
+ *
+ * Readings of points the pages leave open (each one is listed with its
+ * justification in the design notes):
+ *   - Band bounds are inclusive: i - j <= pre and j - i <= next.
+ *   - "Origin at the bottom-right" re-anchors row i at i + (Skv - Sq).
+ *   - mode 5/6: rightDownCausal OR column j < prefix[b] (prefix block is
+ *     anchored at the left edge for every row).
+ *   - mode 7: the last sequence with Sq_b > 0 uses the mode-4 rule, all the
+ *     others the mode-3 rule; mode 8: the first sequence with Sq_b > 0 uses
+ *     the mode-4 rule, all the others the mode-2 rule.
+ *   - Cumulative length arrays hold end offsets without a leading 0.
+ *   - mode 0 without a mask computes everything (pre/next ignored); with a
+ *     mask, the band AND the mask decide.
+ *
+ * Parity status: every function here is pinned by the CPU tests
+ * (tests/test_oracle_pins.py) against library routines, closed forms and the
+ * pages' worked examples. Parity is pinned for all functions.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Layouts of Q/K/V/O (and the matching lse layout). */
+enum { OR_BNSD = 0, OR_BSND = 1, OR_TND = 2 };
+/* Shapes of the optional attenMask. */
+enum { OR_MASK_NONE = 0, OR_MASK_SS = 1, OR_MASK_B1SS = 2, OR_MASK_BNSS = 3 };
+
+typedef struct {
+    int32_t layout;
+    int32_t sparse_mode;
+    int32_t mask_kind;
+    int32_t pad_;
+    int64_t B, N, Sq, Skv, D;     /* TND: Sq, Skv are the token totals */
+    int64_t pre_tokens, next_tokens;
+    double scale;
+} oracle_desc;
+
+/* Per-sequence extents: query/key token offsets and lengths. */
+typedef struct {
+    int64_t q_off, kv_off, sq, skv;
+} seq_info;
+
+static seq_info seq_of(const oracle_desc* d, const int64_t* cu_q,
+                       const int64_t* cu_kv, int64_t b) {
+    seq_info s;
+    if (d->layout == OR_TND) {
+        /* Cumulative ends without a leading 0: {3,5} means lengths 3 and 2. */
+        s.q_off = b == 0 ? 0 : cu_q[b - 1];
+        s.kv_off = b == 0 ? 0 : cu_kv[b - 1];
+        s.sq = cu_q[b] - s.q_off;
+        s.skv = cu_kv[b] - s.kv_off;
+    } else {
+        s.q_off = 0;
+        s.kv_off = 0;
+        s.sq = d->Sq;
+        s.skv = d->Skv;
+    }
+    return s;
+}
+
+/* Band between pre and next, origin at the top-left corner (mode 0). */
+static int band_top_left(int64_t i, int64_t j, int64_t pre, int64_t next) {
+    return (i - j <= pre) && (j - i <= next);
+}
+
+/* Band between pre and next, origin at the bottom-right corner (mode 4):
+ * the row is re-anchored so that the last query row meets the last key. */
+static int band_bottom_right(int64_t i, int64_t j, int64_t sq, int64_t skv,
+                             int64_t pre, int64_t next) {
+    int64_t ir = i + (skv - sq);
+    return (ir - j <= pre) && (j - ir <= next);
+}
+
+/* leftUpCausal: lower triangle split at the top-left vertex (mode 2). */
+static int causal_left_up(int64_t i, int64_t j) { return j <= i; }
+
+/* rightDownCausal: lower triangle split at the bottom-right vertex (mode 3). */
+static int causal_right_down(int64_t i, int64_t j, int64_t sq, int64_t skv) {
+    return j <= i + (skv - sq);
+}
+
+static int64_t mask_index(const oracle_desc* d, int64_t b, int64_t h,
+                          int64_t i, int64_t j) {
+    switch (d->mask_kind) {
+    case OR_MASK_SS:
+        return i * d->Skv + j;
+    case OR_MASK_B1SS:
+        return (b * d->Sq + i) * d->Skv + j;
+    default: /* BNSS */
+        return ((b * d->N + h) * d->Sq + i) * d->Skv + j;
+    }
+}
+
+/* Index of the first / last sequence that has at least one query row. */
+static int64_t first_nonempty(const oracle_desc* d, const int64_t* cu_q,
+                              const int64_t* cu_kv) {
+    for (int64_t b = 0; b < d->B; ++b)
+        if (seq_of(d, cu_q, cu_kv, b).sq > 0) return b;
+    return -1;
+}
+static int64_t last_nonempty(const oracle_desc* d, const int64_t* cu_q,
+                             const int64_t* cu_kv) {
+    for (int64_t b = d->B - 1; b >= 0; --b)
+        if (seq_of(d, cu_q, cu_kv, b).sq > 0) return b;
+    return -1;
+}
+
+/*
+ * Does key j of sequence b contribute to query i of that sequence (head h)?
+ * i and j are positions inside the sequence. One branch per sparseMode
+ * section of the Ascend page.
+ */
+int oracle_visible(const oracle_desc* d, const int64_t* prefix,
+                   const int64_t* cu_q, const int64_t* cu_kv,
+                   const uint8_t* mask, int64_t b, int64_t h, int64_t i,
+                   int64_t j) {
+    seq_info s = seq_of(d, cu_q, cu_kv, b);
+    if (i < 0 || i >= s.sq || j < 0 || j >= s.skv) return 0;
+    switch (d->sparse_mode) {
+    case 0:
+        /* No mask: nothing is masked and pre/next are ignored.
+         * With a mask: the part between pre and next is computed, and a
+         * True mask entry hides its position. */
+        if (mask == NULL || d->mask_kind == OR_MASK_NONE) return 1;
+        if (!band_top_left(i, j, d->pre_tokens, d->next_tokens)) return 0;
+        return mask[mask_index(d, b, h, i, j)] == 0;
+    case 1:
+        /* allMask: the full mask decides; pre/next are ignored. */
+        return mask[mask_index(d, b, h, i, j)] == 0;
+    case 2:
+        return causal_left_up(i, j);
+    case 3:
+        return causal_right_down(i, j, s.sq, s.skv);
+    case 4:
+        return band_bottom_right(i, j, s.sq, s.skv, d->pre_tokens,
+                                 d->next_tokens);
+    case 5:
+    case 6:
+        /* rightDownCausal plus a block Sq long and prefix[b] wide on the
+         * left. */
+        return causal_right_down(i, j, s.sq, s.skv) || (j < prefix[b]);
+    case 7:
+        /* Split from a mode-3 job: the last non-empty sequence is the band. */
+        if (b == last_nonempty(d, cu_q, cu_kv))
+            return band_bottom_right(i, j, s.sq, s.skv, d->pre_tokens,
+                                     d->next_tokens);
+        return causal_right_down(i, j, s.sq, s.skv);
+    case 8:
+        /* Split from a mode-2 job: the first non-empty sequence is the band. */
+        if (b == first_nonempty(d, cu_q, cu_kv))
+            return band_bottom_right(i, j, s.sq, s.skv, d->pre_tokens,
+                                     d->next_tokens);
+        return causal_left_up(i, j);
+    default:
+        return 0;
+    }
+}
+
+/* Element offset of token t (sequence-local position already resolved to a
+ * global row) of head h, batch b, in the given layout. */
+static int64_t row_offset(const oracle_desc* d, int64_t S, int64_t b,
+                          int64_t h, int64_t t) {
+    switch (d->layout) {
+    case OR_BNSD:
+        return ((b * d->N + h) * S + t) * d->D;
+    case OR_BSND:
+        return ((b * S + t) * d->N + h) * d->D;
+    default: /* TND: t is the packed token index */
+        return (t * d->N + h) * d->D;
+    }
+}
+
+static int64_t lse_offset(const oracle_desc* d, int64_t b, int64_t h,
+                          int64_t t) {
+    if (d->layout == OR_TND) return h * d->Sq + t; /* [N, T_q] */
+    return (b * d->N + h) * d->Sq + t;             /* [B, N, Sq] */
+}
+
+/*
+ * One query row of the plain attention definition:
+ *   s_j = scale * sum_d q_d k_jd for the visible j, m = max s_j,
+ *   l = sum exp(s_j - m), o = sum exp(s_j - m) v_j / l, lse = m + ln l.
+ * vis_row holds the explicit visibility of the row's keys.
+ */
+static void attend_row(const oracle_desc* d, const double* q, const double* k,
+                       const double* v, int64_t b, int64_t h, seq_info s,
+                       int64_t i, const uint8_t* vis_row, double* scores,
+                       double* o_row, double* lse_out) {
+    const int64_t D = d->D;
+    const double* qi = q + row_offset(d, d->Sq, b, h, s.q_off + i);
+    double m = -INFINITY;
+    for (int64_t j = 0; j < s.skv; ++j) {
+        if (!vis_row[j]) continue;
+        const double* kj = k + row_offset(d, d->Skv, b, h, s.kv_off + j);
+        double acc = 0.0;
+        for (int64_t x = 0; x < D; ++x) acc += qi[x] * kj[x];
+        scores[j] = d->scale * acc;
+        if (scores[j] > m) m = scores[j];
+    }
+    for (int64_t x = 0; x < D; ++x) o_row[x] = 0.0;
+    if (m == -INFINITY) { /* no visible key */
+        *lse_out = -INFINITY;
+        return;
+    }
+    double l = 0.0;
+    for (int64_t j = 0; j < s.skv; ++j) {
+        if (!vis_row[j]) continue;
+        double p = exp(scores[j] - m);
+        l += p;
+        const double* vj = v + row_offset(d, d->Skv, b, h, s.kv_off + j);
+        for (int64_t x = 0; x < D; ++x) o_row[x] += p * vj[x];
+    }
+    for (int64_t x = 0; x < D; ++x) o_row[x] /= l;
+    *lse_out = m + log(l);
+}
+
+/*
+ * Full forward: O (same layout as Q) and lse for every (b, h, row).
+ * For each (b, h) the explicit Sq_b x Skv_b boolean visibility matrix is
+ * built first, then the plain softmax is applied row by row.
+ */
+int oracle_attn(const oracle_desc* d, const int64_t* prefix,
+                const int64_t* cu_q, const int64_t* cu_kv,
+                const uint8_t* mask, const double* q, const double* k,
+                const double* v, double* o, double* lse) {
+    const int64_t nb = d->B, nh = d->N;
+    int err = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int64_t b = 0; b < nb; ++b) {
+        for (int64_t h = 0; h < nh; ++h) {
+            seq_info s = seq_of(d, cu_q, cu_kv, b);
+            if (s.sq <= 0) continue;
+            int64_t skv_alloc = s.skv > 0 ? s.skv : 1;
+            uint8_t* vis = (uint8_t*)malloc((size_t)(s.sq * skv_alloc));
+            double* scores = (double*)malloc(sizeof(double) * skv_alloc);
+            if (!vis || !scores) {
+                free(vis);
+                free(scores);
+#pragma omp atomic write
+                err = 1;
+                continue;
+            }
+            for (int64_t i = 0; i < s.sq; ++i)
+                for (int64_t j = 0; j < s.skv; ++j)
+                    vis[i * skv_alloc + j] = (uint8_t)oracle_visible(
+                        d, prefix, cu_q, cu_kv, mask, b, h, i, j);
+            for (int64_t i = 0; i < s.sq; ++i) {
+                double* o_row = o + row_offset(d, d->Sq, b, h, s.q_off + i);
+                attend_row(d, q, k, v, b, h, s, i, vis + i * skv_alloc,
+                           scores, o_row, lse + lse_offset(d, b, h, s.q_off + i));
+            }
+            free(vis);
+            free(scores);
+        }
+    }
+    return err;
+}
+
+/*
+ * Selected rows only, for spot checks of large problems: rows[3*r + 0..2] =
+ * (b, h, i) with i the position inside sequence b. o_rows is [nrows, D].
+ */
+int oracle_attn_rows(const oracle_desc* d, const int64_t* prefix,
+                     const int64_t* cu_q, const int64_t* cu_kv,
+                     const uint8_t* mask, const double* q, const double* k,
+                     const double* v, int64_t nrows, const int64_t* rows,
+                     double* o_rows, double* lse_rows) {
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+        seq_info s = seq_of(d, cu_q, cu_kv, b);
+        int64_t skv_alloc = s.skv > 0 ? s.skv : 1;
+        uint8_t* vis = (uint8_t*)malloc((size_t)skv_alloc);
+        double* scores = (double*)malloc(sizeof(double) * skv_alloc);
+        if (!vis || !scores) {
+            free(vis);
+            free(scores);
+#pragma omp atomic write
+            err = 1;
+            continue;
+        }
+        for (int64_t j = 0; j < s.skv; ++j)
+            vis[j] = (uint8_t)oracle_visible(d, prefix, cu_q, cu_kv, mask, b,
+                                             h, i, j);
+        attend_row(d, q, k, v, b, h, s, i, vis, scores, o_rows + r * d->D,
+                   lse_rows + r);
+        free(vis);
+        free(scores);
+    }
+    return err;
+}
+
+/* Explicit visibility matrix of sequence b, head h: out is [Sq_b, Skv_b]. */
+void oracle_mask(const oracle_desc* d, const int64_t* prefix,
+                 const int64_t* cu_q, const int64_t* cu_kv,
+                 const uint8_t* mask, int64_t b, int64_t h, uint8_t* out) {
+    seq_info s = seq_of(d, cu_q, cu_kv, b);
+    for (int64_t i = 0; i < s.sq; ++i)
+        for (int64_t j = 0; j < s.skv; ++j)
+            out[i * s.skv + j] = (uint8_t)oracle_visible(d, prefix, cu_q,
+                                                         cu_kv, mask, b, h, i, j);
+}
+
+/* Number of visible (b, h, i, j) pairs, by enumeration. */
+int64_t oracle_visible_count(const oracle_desc* d, const int64_t* prefix,
+                             const int64_t* cu_q, const int64_t* cu_kv,
+                             const uint8_t* mask) {
+    int64_t total = 0;
+    const int64_t nb = d->B, nh = d->N;
+#pragma omp parallel for collapse(2) reduction(+ : total) schedule(dynamic, 1)
+    for (int64_t b = 0; b < nb; ++b) {
+        for (int64_t h = 0; h < nh; ++h) {
+            seq_info s = seq_of(d, cu_q, cu_kv, b);
+            int64_t c = 0;
+            for (int64_t i = 0; i < s.sq; ++i)
+                for (int64_t j = 0; j < s.skv; ++j)
+                    c += oracle_visible(d, prefix, cu_q, cu_kv, mask, b, h, i, j);
+            total += c;
+        }
+    }
+    return total;
+}
+
+/*
+ * The exercise page's tiled CPU attention, in the page's normalised form.
+ * q, k, v, out are [B, S, D]; keys are visited in blocks of `block` (the
+ * last block may be shorter). vis (optional, [B, S, S], 1 = visible) masks
+ * keys; a block with no visible key for a row leaves that row's state as it
+ * was. For each block:
+ *   m_new = max(m_old, m_blk)
+ *   l_new = l_old e^(m_old - m_new) + sum_j e^(s_j - m_new)
+ *   O_new = (O_old l_old e^(m_old - m_new) + sum_j e^(s_j - m_new) v_j) / l_new
+ */
+void oracle_flash_tiled(const double* q, const double* k, const double* v,
+                        const uint8_t* vis, int64_t B, int64_t S, int64_t D,
+                        int64_t block, double scale, double* out) {
+    double* s_blk = (double*)malloc(sizeof(double) * (size_t)block);
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t i = 0; i < S; ++i) {
+            const double* qi = q + (b * S + i) * D;
+            double* oi = out + (b * S + i) * D;
+            double m_old = -INFINITY, l_old = 0.0;
+            for (int64_t x = 0; x < D; ++x) oi[x] = 0.0;
+            for (int64_t j0 = 0; j0 < S; j0 += block) {
+                int64_t j1 = j0 + block < S ? j0 + block : S;
+                double m_blk = -INFINITY;
+                for (int64_t j = j0; j < j1; ++j) {
+                    if (vis && !vis[(b * S + i) * S + j]) {
+                        s_blk[j - j0] = -INFINITY;
+                        continue;
+                    }
+                    const double* kj = k + (b * S + j) * D;
+                    double acc = 0.0;
+                    for (int64_t x = 0; x < D; ++x) acc += qi[x] * kj[x];
+                    s_blk[j - j0] = scale * acc;
+                    if (s_blk[j - j0] > m_blk) m_blk = s_blk[j - j0];
+                }
+                if (m_blk == -INFINITY) continue; /* nothing visible here */
+                double m_new = m_old > m_blk ? m_old : m_blk;
+                double carry = (m_old == -INFINITY) ? 0.0 : exp(m_old - m_new);
+                double l_new = l_old * carry;
+                for (int64_t j = j0; j < j1; ++j)
+                    if (s_blk[j - j0] != -INFINITY) l_new += exp(s_blk[j - j0] - m_new);
+                for (int64_t x = 0; x < D; ++x) {
+                    double acc = oi[x] * l_old * carry;
+                    for (int64_t j = j0; j < j1; ++j)
+                        if (s_blk[j - j0] != -INFINITY)
+                            acc += exp(s_blk[j - j0] - m_new) * v[(b * S + j) * D + x];
+                    oi[x] = acc / l_new;
+                }
+                m_old = m_new;
+                l_old = l_new;
+            }
+        }
+    }
+    free(s_blk);
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
