@@ -1,0 +1,382 @@
+"""Benchmark of the B200 masked attention forward.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference] [--workload NAME]
+
+Prints ONE JSON line (rank 0). A step is one fa_fwd over the whole workload
+(every KV tile of every (sequence, head, query block)). The metric counts
+only visible (i, j) pairs: TFLOP/s = 4 * D * pairs / time.
+
+Default workload: B=2, N=16, Sq=Skv=4096, D=128, BNSD, sparseMode 2
+(leftUpCausal), bf16 N(0,1) inputs from seed 2. With --gpus N > 1 (under
+torchrun) every rank runs its own independent copy of the workload (the
+work shards by (batch, head, query block) with no exchange), so the value
+is the total over ranks divided by the slowest rank's time (weak scaling).
+
+Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events
+on the launching stream; a 256 MiB buffer (larger than the 126 MB L2) is
+written between steps, outside the events, so every step starts with a cold
+L2. Barrier + synchronize on both sides of the timed region, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "leftup_causal_4k"
+METRIC = "masked-attention fwd TFLOP/s (visible pairs) and % of B200 BF16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="budget of the oracle's bounded CPU sample")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(workload):
+    """Per-launch DRAM bytes of the main kernel from the committed ncu summary."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            return json.load(f).get(workload)
+    except (OSError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def workload_args(w):
+    import numpy as np
+    arrays = {}
+    if w.prefix is not None:
+        arrays["prefix"] = np.asarray(w.prefix, dtype=np.int64)
+    if w.layout == "TND":
+        arrays["actual_seq_qlen"] = np.asarray(w.actual_seq_qlen, dtype=np.int64)
+        arrays["actual_seq_kvlen"] = np.asarray(w.actual_seq_kvlen, dtype=np.int64)
+    return arrays
+
+
+def visible_pairs(w, has_mask, mask_host=None):
+    """Visible pairs of the workload from the library's geometry (closed-form
+    row intervals); dense-mask workloads count the mask on the host."""
+    import masked_attention_fa_b200 as fa
+    if has_mask:
+        import numpy as np
+        import torch
+        m = mask_host.to(torch.bool).numpy()
+        S = w.Sq
+        ii = np.arange(S)[:, None]
+        jj = np.arange(w.Skv)[None, :]
+        band = (ii - jj <= w.pre_tokens) & (jj - ii <= w.next_tokens)
+        per = int(((~m) & band).sum()) if m.ndim == 2 else int(((~m) & band).sum())
+        return per * (w.N * w.B if m.ndim == 2 else 1)
+    d = fa.make_desc(w.layout, w.B, w.N, w.Sq, w.Skv, w.D, w.sparse_mode, w.pre_tokens,
+                     w.next_tokens, w.scale, w.mask_kind)
+    return fa.fa_visible_pairs(d, **workload_args(w))
+
+
+def cpu_baseline_sample(w, inputs, seconds):
+    """Time the oracle (as it stands) on a bounded sample of query rows of the
+    same workload; returns (TFLOP/s, cores, description)."""
+    import numpy as np
+    import oracle
+    from oracle import Problem
+    pb_kw = dict(layout=w.layout, B=w.B, N=w.N, Sq=w.Sq, Skv=w.Skv, D=w.D,
+                 sparse_mode=w.sparse_mode, pre_tokens=w.pre_tokens, next_tokens=w.next_tokens,
+                 scale=w.scale)
+    # One (batch, head) slice, converted once; rows sampled evenly.
+    b, h = 0, 0
+    q, k, v = inputs["q"], inputs["k"], inputs["v"]
+    if w.layout == "BNSD":
+        qs, ks, vs = q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1]
+        sub = dict(pb_kw, B=1, N=1)
+    elif w.layout == "BSND":
+        qs, ks, vs = q[b:b + 1, :, h:h + 1], k[b:b + 1, :, h:h + 1], v[b:b + 1, :, h:h + 1]
+        sub = dict(pb_kw, B=1, N=1)
+    else:
+        qs, ks, vs = q[:, h:h + 1], k[:, h:h + 1], v[:, h:h + 1]
+        sub = dict(pb_kw, N=1, actual_seq_qlen=w.actual_seq_qlen,
+                   actual_seq_kvlen=w.actual_seq_kvlen)
+    if w.prefix is not None:
+        sub["prefix"] = [w.prefix[b]] if w.layout != "TND" else w.prefix
+    mask = inputs.get("mask")
+    if mask is not None:
+        sub["mask"] = mask.numpy()
+        sub["mask_kind"] = w.mask_kind
+    pb = Problem(**sub)
+    qd, kd, vd = (oracle._f64(x.contiguous()) for x in (qs, ks, vs))
+    nrows_total = w.Sq if w.layout != "TND" else w.actual_seq_qlen[0]
+    row_pairs = oracle.mask_matrix(pb, 0).sum(axis=1, dtype=np.int64)
+    done_rows, pairs, elapsed, chunk = 0, 0, 0.0, 64
+    rng = np.random.default_rng(0)
+    while elapsed < seconds and done_rows < 1_000_000:
+        rows_i = rng.integers(0, nrows_total, size=chunk)
+        rows = np.stack([np.zeros(chunk, np.int64), np.zeros(chunk, np.int64), rows_i], 1)
+        t0 = time.perf_counter()
+        oracle.attention_rows(pb, qd, kd, vd, rows)
+        elapsed += time.perf_counter() - t0
+        pairs += int(row_pairs[rows_i].sum())
+        done_rows += chunk
+        chunk = min(chunk * 2, 4096)
+    tflops = 4.0 * w.D * pairs / elapsed / 1e12
+    desc = (f"{done_rows} query rows drawn uniformly from batch 0, head 0 of {w.name}; "
+            f"{pairs} visible pairs in {elapsed:.1f} s")
+    return tflops, oracle.num_threads(), desc
+
+
+def run_reference(args):
+    """The oracle on the host cores, as the reference arm."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from masked_attention_fa_b200.workloads import named_workloads, make_inputs
+    import oracle
+    w = named_workloads()[args.workload]
+    inputs = make_inputs(w)
+    per_step = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    desc = None
+    cores = oracle.num_threads()
+    for s in range(args.warmup + args.steps):
+        tf, cores, desc = cpu_baseline_sample(w, inputs, per_step)
+        if s >= args.warmup:
+            vals.append(tf)
+    value = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name, "layout": w.layout, "B": w.B,
+                                            "N": w.N, "Sq": w.Sq, "Skv": w.Skv, "D": w.D,
+                                            "sparse_mode": w.sparse_mode},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import masked_attention_fa_b200 as fa
+    from masked_attention_fa_b200.workloads import named_workloads, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    w = named_workloads()[args.workload]
+    inputs = make_inputs(w)
+    q, k, v = (inputs[x].to(dev) for x in ("q", "k", "v"))
+    mask = inputs["mask"].to(dev) if inputs["mask"] is not None else None
+    arrays = workload_args(w)
+    attn = fa.MaskedAttention(w.layout, w.B, w.N, w.Sq, w.Skv, w.D, w.sparse_mode, w.pre_tokens,
+                              w.next_tokens, w.scale, w.mask_kind)
+    oshape, lshape = attn.out_shapes()
+    o = torch.empty(oshape, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(lshape, dtype=torch.float32, device=dev)
+    pairs = visible_pairs(w, mask is not None, inputs["mask"])
+    flops = 4.0 * w.D * pairs
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        attn(q, k, v, atten_mask=mask, out=o, lse=lse, stream=stream, **arrays)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    attn.sync_status()
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    attn.sync_status()
+    times_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = sum(times_ms) / len(times_ms)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    value = world * flops / (ms_max * 1e-3) / 1e12
+
+    # End to end through the public API with host buffers: pinned host
+    # inputs -> device, forward, O and lse -> pinned host, every step.
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (x.pin_memory() for x in (inputs["q"], inputs["k"], inputs["v"]))
+        ho = torch.empty(oshape, dtype=torch.bfloat16).pin_memory()
+        hl = torch.empty(lshape, dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 10))
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = e0.elapsed_time(e1) / n_e2e
+        te = torch.tensor([ems], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * flops / (float(te.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(sum(x.numel() * x.element_size() for x in (hq, hk, hv))),
+               "d2h_bytes_per_step": int(ho.numel() * ho.element_size() +
+                                         hl.numel() * hl.element_size())}
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        peak = float(peaks["bf16_tflops"])
+        achieved = flops / (ms * 1e-3) / 1e12
+        traffic = load_traffic(w.name)
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": traffic,
+                    "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
+                    "kernel": f"fa_fwd_sm100<{w.D}>"}
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            tf, cores, desc = cpu_baseline_sample(w, inputs, args.cpu_seconds)
+            cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                   "sample": desc}
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": w.name, "layout": w.layout, "B": w.B, "N": w.N,
+                           "Sq": w.Sq, "Skv": w.Skv, "D": w.D, "sparse_mode": w.sparse_mode,
+                           "visible_pairs": pairs, "per_rank": "independent copy",
+                           "l2": "256 MiB buffer written between timed steps (cold L2)",
+                           "parallelism": f"replicas x{world}"},
+                "frac_of_peak": value / world / peak,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": args.steps, "clocks": clocks,
+                "ms_min": min(times_ms), "ms_median": statistics.median(times_ms)}
+        print(json.dumps(line))
+    attn.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,204 @@
+/*
+ * fa.h — C ABI of the B200 (sm_100a) masked attention forward.
+ *
+ *   O = softmax(scale * Q K^T masked by the sparseMode geometry) V
+ *
+ * computed tile by tile with an online softmax (running row max m_i and
+ * running row sum l_i), never materialising the Sq x Skv score matrix.
+ * Operation: the "FlashAttention tiling & online softmax" exercise page
+ * (section "Mục tiêu kiến thức": running maximum m_i, running sum l_i).
+ * Mask geometry: the Ascend CANN page "sparseMode参数说明", sections
+ * sparseMode=0 .. sparseMode=8, and its attenMask rule (a True entry hides
+ * the QK^T position).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Two stages, as the aclnnScatterPaKvCache page's host flow does: a
+ *    descriptor is validated and turned into a handle once (fa_create),
+ *    then the handle runs calls on a caller-supplied CUDA stream (fa_fwd).
+ *  - All validation happens on the host before any device work; a call that
+ *    returns a non-OK status has touched no output and enqueued nothing.
+ *    fa_last_error() then returns a message for the calling thread.
+ *  - Status codes follow the null-pointer / invalid-parameter split of the
+ *    aclnnScatterPaKvCache page's "返回值" table.
+ *  - Results are bitwise deterministic: every output row is produced by one
+ *    CTA, visiting its key tiles in a fixed order (no split-K atomics), as
+ *    the aclnnScatterPaKvCache page's "确定性计算" note asks of that op.
+ *  - A handle is not thread-safe; distinct handles are independent.
+ */
+#ifndef FA_B200_FA_H
+#define FA_B200_FA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FA_VERSION 1
+
+typedef struct fa_handle_s* fa_handle_t;
+
+/* Memory layouts of Q, K, V and O (bf16, dense, innermost dimension D):
+ *   FA_BNSD  Q/O [B, N, Sq, D],  K/V [B, N, Skv, D]
+ *   FA_BSND  Q/O [B, Sq, N, D],  K/V [B, Skv, N, D]
+ *   FA_TND   Q/O [T_q, N, D],    K/V [T_kv, N, D]  (varlen, packed tokens)
+ * lse is fp32 [B, N, Sq] for BNSD/BSND and [N, T_q] for TND. */
+typedef enum { FA_BNSD = 0, FA_BSND = 1, FA_TND = 2 } fa_layout_t;
+
+/* Shapes of the optional attenMask (uint8, nonzero = masked), read only in
+ * sparseMode 0 and 1:  SS [Sq, Skv], B1SS [B, 1, Sq, Skv], BNSS [B, N, Sq, Skv]. */
+typedef enum {
+    FA_MASK_NONE = 0,
+    FA_MASK_SS = 1,
+    FA_MASK_B1SS = 2,
+    FA_MASK_BNSS = 3
+} fa_mask_kind_t;
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_NULLPTR = 1,        /* a required pointer is NULL */
+    FA_ERR_PARAM_INVALID = 2,  /* a value breaks a documented constraint */
+    FA_ERR_SHAPE = 3,          /* sizes or length arrays are inconsistent */
+    FA_ERR_UNSUPPORTED = 4,    /* valid request outside this build (e.g. D) */
+    FA_ERR_ALLOC = 5,          /* host or device allocation failed */
+    FA_ERR_CUDA = 6,           /* a CUDA runtime call failed */
+    FA_ERR_TIMEOUT = 7,        /* a device-side wait gave up (kernel aborted) */
+    FA_ERR_DEVICE = 8          /* the kernel reported an internal error */
+} fa_status_t;
+
+/* Problem descriptor. For FA_TND, B is the number of sequences and Sq / Skv
+ * are the token totals T_q / T_kv. */
+typedef struct {
+    int32_t layout;        /* fa_layout_t */
+    int32_t sparse_mode;   /* 0..8 */
+    int32_t mask_kind;     /* fa_mask_kind_t; must be NONE unless mode 0/1 */
+    int32_t reserved;      /* must be 0 */
+    int64_t B, N, Sq, Skv, D;
+    int64_t pre_tokens;    /* preTokens  (modes 0, 4, 7, 8; ignored otherwise) */
+    int64_t next_tokens;   /* nextTokens (modes 0, 4, 7, 8; ignored otherwise) */
+    double scale;          /* multiplies q.k before the softmax; > 0, finite */
+} fa_desc_t;
+
+/*
+ * fa_create — validate the static part of a descriptor and make a handle.
+ *
+ * desc: host pointer, read during the call only. out: receives the handle.
+ * Constraints checked here (the rest needs the per-call arrays, see fa_fwd):
+ *   layout in {BNSD, BSND, TND}; sparse_mode in 0..8; B, N, D >= 1;
+ *   Sq, Skv >= 0 and < 2^30; D in {64, 128} (FA_ERR_UNSUPPORTED otherwise);
+ *   scale finite and > 0; mask_kind is NONE for modes 2..8; mode 1 needs a
+ *   mask kind; a mask with TND is FA_ERR_UNSUPPORTED (the sparseMode page
+ *   gives no TND mask shape); modes 7 and 8 need TND; in mode 0 with a mask,
+ *   next < 0 needs pre >= |next| and |next| < Skv, pre < 0 needs
+ *   next >= |pre| and |pre| < Sq (sparseMode=0 section, the two 说明 notes);
+ *   in mode 4 the band must intersect: pre + next >= 0 (sparseMode=4).
+ * Ownership: the handle owns a small device workspace (work list, counters,
+ * error word) and a pinned staging buffer, released by fa_destroy. The
+ * workspace is allocated on the current device at the first fa_fwd.
+ */
+fa_status_t fa_create(const fa_desc_t* desc, fa_handle_t* out);
+
+/*
+ * fa_fwd — enqueue one masked attention forward on `cuda_stream`.
+ *
+ * q, k, v      device, bf16, dense in the handle's layout; 16-byte aligned.
+ * atten_mask   device uint8 in the handle's mask_kind shape, nonzero =
+ *              masked; read in modes 0 and 1 only (NULL in mode 0 means
+ *              "no mask": nothing is masked and pre/next are ignored, as the
+ *              sparseMode=0 section states). Ignored for modes 2..8.
+ * prefix       host int64[B]; modes 5/6 only: prefix[b] leading key columns
+ *              are visible to every query row of batch b; 0 <= prefix[b] <=
+ *              Skv_b.
+ * actual_seq_qlen, actual_seq_kvlen
+ *              host int64[B], TND only: cumulative end offsets without a
+ *              leading 0 ({3,5} means lengths 3 and 2), non-decreasing, last
+ *              entries equal to Sq and Skv of the descriptor.
+ * o            device bf16, same layout and shape as q.
+ * lse          device fp32, natural-log sum of exp(scale q.k) over the
+ *              visible keys of each row; -inf (and O = 0) for a row with no
+ *              visible key.
+ * cuda_stream  a cudaStream_t (NULL = legacy default stream).
+ *
+ * Per-call constraints (sparseMode=7/8 sections): mode 7 needs, for the last
+ * sequence with Sq_b > 0: pre >= Skv_b and Sq_b - Skv_b <= next <= 0, and
+ * Sq_b <= Skv_b for every other sequence; mode 8 needs, for the first
+ * sequence with Sq_b > 0: pre >= Skv_b and next >= Sq_b - Skv_b. Violations
+ * return FA_ERR_PARAM_INVALID before any device work.
+ *
+ * Asynchronous: returns once the kernel is enqueued. The host arrays are
+ * read during the call only. Device-side problems (a wait that gave up) are
+ * reported by fa_sync_status. The device must be sm_100 (B200 class);
+ * otherwise FA_ERR_UNSUPPORTED.
+ */
+fa_status_t fa_fwd(fa_handle_t h, const void* q, const void* k, const void* v,
+                   const uint8_t* atten_mask, const int64_t* prefix,
+                   const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
+                   void* o, float* lse, void* cuda_stream);
+
+/* fa_sync_status — wait for the handle's last call and read its device error
+ * word: FA_OK, FA_ERR_TIMEOUT (a bounded wait in the kernel gave up, its
+ * outputs are undefined) or FA_ERR_DEVICE. The error word is cleared. */
+fa_status_t fa_sync_status(fa_handle_t h);
+
+/* fa_destroy — wait for the handle's work and free everything it owns.
+ * NULL is accepted. */
+fa_status_t fa_destroy(fa_handle_t h);
+
+/* Message of the calling thread's last non-OK status ("" if none). Valid
+ * until the thread's next fa_* call. */
+const char* fa_last_error(void);
+
+/* Library version (FA_VERSION). */
+int32_t fa_version(void);
+
+/* ---------------- host-only helpers (no device work) ------------------- */
+
+/*
+ * fa_validate — every check that fa_create and fa_fwd make, without a
+ * handle and without touching any device. has_mask: whether atten_mask would
+ * be non-NULL. Arrays as in fa_fwd (host).
+ */
+fa_status_t fa_validate(const fa_desc_t* desc, const int64_t* prefix,
+                        const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
+                        int32_t has_mask);
+
+/*
+ * fa_visible_pairs — number of visible (b, h, i, j) pairs of a valid call,
+ * from the closed-form row intervals of the geometry (the FLOP count of the
+ * throughput metric is 4 * D * pairs). Modes with a dense mask (mode 1, mode 0
+ * with a mask) are FA_ERR_UNSUPPORTED: their count depends on the mask data.
+ */
+fa_status_t fa_visible_pairs(const fa_desc_t* desc, const int64_t* prefix,
+                             const int64_t* actual_seq_qlen,
+                             const int64_t* actual_seq_kvlen, int32_t has_mask,
+                             int64_t* pairs_out);
+
+/* Tile classes of the scheduler (tiles are 128 query rows x 128 keys). */
+typedef enum { FA_TILE_EMPTY = 0, FA_TILE_PARTIAL = 1, FA_TILE_FULL = 2 } fa_tile_class_t;
+
+/*
+ * fa_tile_class — how the scheduler classifies the tile of sequence b with
+ * query rows [128 qt, 128 qt + 128) and keys [128 kt, 128 kt + 128) (rows and
+ * keys inside the sequence): EMPTY tiles are skipped, PARTIAL tiles get an
+ * element mask, FULL tiles none. Returns the class, or -1 on invalid input.
+ */
+int32_t fa_tile_class(const fa_desc_t* desc, const int64_t* prefix,
+                      const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
+                      int32_t has_mask, int64_t b, int64_t qt, int64_t kt);
+
+/*
+ * fa_plan_stats — size of the work list a call would run: out[0] = work
+ * items (one per (sequence, head, block of 256 query rows) with at least one
+ * query row), out[1] = EMPTY, out[2] = PARTIAL, out[3] = FULL 128x128 tiles
+ * over all items and heads. out: host int64[4].
+ */
+fa_status_t fa_plan_stats(const fa_desc_t* desc, const int64_t* prefix,
+                          const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
+                          int32_t has_mask, int64_t* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_FA_H */

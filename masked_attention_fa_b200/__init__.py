@@ -1,0 +1,261 @@
+"""Python binding of the B200 masked attention forward C ABI (include/fa.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library ``libfa_b200.so`` (built in-tree by ``masked_attention_fa_b200.build``).
+PyTorch is used for device memory and streams. If the library is missing the
+import of any entry point fails loudly; there is no fallback.
+
+The C entry points keep their names (``fa_create``, ``fa_fwd``, ...). The
+``MaskedAttention`` class wraps a handle for convenience.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa_b200.so")
+
+FA_BNSD, FA_BSND, FA_TND = 0, 1, 2
+LAYOUTS = {"BNSD": FA_BNSD, "BSND": FA_BSND, "TND": FA_TND}
+FA_MASK_NONE, FA_MASK_SS, FA_MASK_B1SS, FA_MASK_BNSS = 0, 1, 2, 3
+MASK_KINDS = {None: FA_MASK_NONE, "SS": FA_MASK_SS, "B1SS": FA_MASK_B1SS, "BNSS": FA_MASK_BNSS}
+STATUS = {0: "FA_OK", 1: "FA_ERR_NULLPTR", 2: "FA_ERR_PARAM_INVALID", 3: "FA_ERR_SHAPE",
+          4: "FA_ERR_UNSUPPORTED", 5: "FA_ERR_ALLOC", 6: "FA_ERR_CUDA", 7: "FA_ERR_TIMEOUT",
+          8: "FA_ERR_DEVICE"}
+FA_TILE_EMPTY, FA_TILE_PARTIAL, FA_TILE_FULL = 0, 1, 2
+
+
+class FaError(RuntimeError):
+    def __init__(self, status, message):
+        self.status = status
+        self.name = STATUS.get(status, str(status))
+        super().__init__(f"{self.name}: {message}")
+
+
+class fa_desc_t(ctypes.Structure):
+    _fields_ = [
+        ("layout", ctypes.c_int32),
+        ("sparse_mode", ctypes.c_int32),
+        ("mask_kind", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("B", ctypes.c_int64),
+        ("N", ctypes.c_int64),
+        ("Sq", ctypes.c_int64),
+        ("Skv", ctypes.c_int64),
+        ("D", ctypes.c_int64),
+        ("pre_tokens", ctypes.c_int64),
+        ("next_tokens", ctypes.c_int64),
+        ("scale", ctypes.c_double),
+    ]
+
+
+_lib = None
+
+
+def load_library():
+    """Load libfa_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m masked_attention_fa_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    dp = ctypes.POINTER(fa_desc_t)
+    st = ctypes.c_int32
+    lib.fa_create.argtypes = [dp, ctypes.POINTER(P)]
+    lib.fa_create.restype = st
+    lib.fa_fwd.argtypes = [P, P, P, P, P, i64p, i64p, i64p, P, P, P]
+    lib.fa_fwd.restype = st
+    lib.fa_sync_status.argtypes = [P]
+    lib.fa_sync_status.restype = st
+    lib.fa_destroy.argtypes = [P]
+    lib.fa_destroy.restype = st
+    lib.fa_last_error.argtypes = []
+    lib.fa_last_error.restype = ctypes.c_char_p
+    lib.fa_version.argtypes = []
+    lib.fa_version.restype = ctypes.c_int32
+    lib.fa_validate.argtypes = [dp, i64p, i64p, i64p, ctypes.c_int32]
+    lib.fa_validate.restype = st
+    lib.fa_visible_pairs.argtypes = [dp, i64p, i64p, i64p, ctypes.c_int32, i64p]
+    lib.fa_visible_pairs.restype = st
+    lib.fa_tile_class.argtypes = [dp, i64p, i64p, i64p, ctypes.c_int32, ctypes.c_int64,
+                                  ctypes.c_int64, ctypes.c_int64]
+    lib.fa_tile_class.restype = ctypes.c_int32
+    lib.fa_plan_stats.argtypes = [dp, i64p, i64p, i64p, ctypes.c_int32, i64p]
+    lib.fa_plan_stats.restype = st
+    _lib = lib
+    return lib
+
+
+EXPORTED = ("fa_create", "fa_fwd", "fa_sync_status", "fa_destroy", "fa_last_error",
+            "fa_version", "fa_validate", "fa_visible_pairs", "fa_tile_class", "fa_plan_stats")
+
+
+def _check(status):
+    if status != 0:
+        msg = load_library().fa_last_error().decode(errors="replace")
+        raise FaError(status, msg)
+
+
+def make_desc(layout, B, N, Sq, Skv, D, sparse_mode=0, pre_tokens=0, next_tokens=0, scale=None,
+              mask_kind=None) -> fa_desc_t:
+    lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+    mk = MASK_KINDS[mask_kind] if (mask_kind is None or isinstance(mask_kind, str)) else int(mask_kind)
+    sc = (1.0 / float(D) ** 0.5) if scale is None else float(scale)
+    return fa_desc_t(lay, int(sparse_mode), mk, 0, int(B), int(N), int(Sq), int(Skv), int(D),
+                     int(pre_tokens), int(next_tokens), sc)
+
+
+class _Arrays:
+    """Host int64 arrays for prefix / actual_seq_* kept alive for one call."""
+
+    def __init__(self, prefix, cu_q, cu_kv):
+        self.prefix = None if prefix is None else np.ascontiguousarray(prefix, dtype=np.int64)
+        self.cu_q = None if cu_q is None else np.ascontiguousarray(cu_q, dtype=np.int64)
+        self.cu_kv = None if cu_kv is None else np.ascontiguousarray(cu_kv, dtype=np.int64)
+
+    @staticmethod
+    def _p(a):
+        if a is None:
+            return None
+        return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+
+    def ptrs(self):
+        return self._p(self.prefix), self._p(self.cu_q), self._p(self.cu_kv)
+
+
+# ---------------------------------------------------------------- C names
+
+def fa_version() -> int:
+    return int(load_library().fa_version())
+
+
+def fa_last_error() -> str:
+    return load_library().fa_last_error().decode(errors="replace")
+
+
+def fa_validate(desc, prefix=None, actual_seq_qlen=None, actual_seq_kvlen=None, has_mask=False):
+    """Status code of the host-side checks (0 = valid)."""
+    a = _Arrays(prefix, actual_seq_qlen, actual_seq_kvlen)
+    return int(load_library().fa_validate(ctypes.byref(desc), *a.ptrs(), int(bool(has_mask))))
+
+
+def fa_visible_pairs(desc, prefix=None, actual_seq_qlen=None, actual_seq_kvlen=None,
+                     has_mask=False) -> int:
+    a = _Arrays(prefix, actual_seq_qlen, actual_seq_kvlen)
+    out = ctypes.c_int64(0)
+    _check(load_library().fa_visible_pairs(ctypes.byref(desc), *a.ptrs(), int(bool(has_mask)),
+                                           ctypes.byref(out)))
+    return int(out.value)
+
+
+def fa_tile_class(desc, b, qt, kt, prefix=None, actual_seq_qlen=None, actual_seq_kvlen=None,
+                  has_mask=False) -> int:
+    a = _Arrays(prefix, actual_seq_qlen, actual_seq_kvlen)
+    return int(load_library().fa_tile_class(ctypes.byref(desc), *a.ptrs(), int(bool(has_mask)),
+                                             int(b), int(qt), int(kt)))
+
+
+def fa_plan_stats(desc, prefix=None, actual_seq_qlen=None, actual_seq_kvlen=None,
+                  has_mask=False):
+    """(work items, EMPTY, PARTIAL, FULL) of the scheduler for one call."""
+    a = _Arrays(prefix, actual_seq_qlen, actual_seq_kvlen)
+    out = (ctypes.c_int64 * 4)()
+    _check(load_library().fa_plan_stats(ctypes.byref(desc), *a.ptrs(), int(bool(has_mask)), out))
+    return tuple(int(x) for x in out)
+
+
+def fa_create(desc) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(load_library().fa_create(ctypes.byref(desc), ctypes.byref(h)))
+    return h
+
+
+def fa_destroy(h):
+    _check(load_library().fa_destroy(h))
+
+
+def fa_sync_status(h) -> int:
+    """Raw status of the handle's last call (0 = OK)."""
+    return int(load_library().fa_sync_status(h))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def fa_fwd(h, q, k, v, o, lse, atten_mask=None, prefix=None, actual_seq_qlen=None,
+           actual_seq_kvlen=None, stream=None):
+    """Enqueue one forward on `stream` (torch.cuda.Stream, raw handle int, or
+    None = torch's current stream). Tensors must be CUDA tensors."""
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    elif hasattr(stream, "cuda_stream"):
+        stream = stream.cuda_stream
+    a = _Arrays(prefix, actual_seq_qlen, actual_seq_kvlen)
+    _check(load_library().fa_fwd(h, _ptr(q), _ptr(k), _ptr(v), _ptr(atten_mask), *a.ptrs(),
+                                 _ptr(o), _ptr(lse), ctypes.c_void_p(int(stream))))
+
+
+# ---------------------------------------------------------------- helper class
+
+class MaskedAttention:
+    """A handle for one problem shape: ``o, lse = attn(q, k, v, ...)``."""
+
+    def __init__(self, layout, B, N, Sq, Skv, D, sparse_mode=0, pre_tokens=0, next_tokens=0,
+                 scale=None, mask_kind=None):
+        self.layout = layout
+        self.desc = make_desc(layout, B, N, Sq, Skv, D, sparse_mode, pre_tokens, next_tokens,
+                              scale, mask_kind)
+        self.handle = fa_create(self.desc)
+
+    def out_shapes(self):
+        d = self.desc
+        if self.layout == "BNSD":
+            return (d.B, d.N, d.Sq, d.D), (d.B, d.N, d.Sq)
+        if self.layout == "BSND":
+            return (d.B, d.Sq, d.N, d.D), (d.B, d.N, d.Sq)
+        return (d.Sq, d.N, d.D), (d.N, d.Sq)
+
+    def __call__(self, q, k, v, atten_mask=None, prefix=None, actual_seq_qlen=None,
+                 actual_seq_kvlen=None, out=None, lse=None, stream=None):
+        import torch
+        oshape, lshape = self.out_shapes()
+        if out is None:
+            out = torch.empty(oshape, dtype=torch.bfloat16, device=q.device)
+        if lse is None:
+            lse = torch.empty(lshape, dtype=torch.float32, device=q.device)
+        for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+            if t.dtype != torch.bfloat16 or not t.is_contiguous() or not t.is_cuda:
+                raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+        if not lse.is_contiguous() or lse.dtype != torch.float32:
+            raise ValueError("lse must be a contiguous fp32 tensor")
+        if atten_mask is not None:
+            if atten_mask.dtype not in (torch.uint8, torch.bool) or not atten_mask.is_contiguous():
+                raise ValueError("atten_mask must be a contiguous uint8/bool tensor")
+        fa_fwd(self.handle, q, k, v, out, lse, atten_mask, prefix, actual_seq_qlen,
+               actual_seq_kvlen, stream)
+        return out, lse
+
+    def sync_status(self):
+        st = fa_sync_status(self.handle)
+        if st != 0:
+            raise FaError(st, fa_last_error())
+
+    def close(self):
+        if self.handle is not None:
+            fa_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

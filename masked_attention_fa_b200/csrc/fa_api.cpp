@@ -1,0 +1,341 @@
+// C ABI front end: handles, per-call plan caching and the kernel launch.
+//
+// Two-stage use as the aclnnScatterPaKvCache page's host flow describes it:
+// the descriptor is checked once (fa_create), then each fa_fwd validates its
+// per-call arrays, reuses or rebuilds the cached work list, copies it to the
+// handle's device workspace through pinned staging memory and enqueues the
+// persistent kernel on the caller's stream.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/fa.h"
+#include "fa_kernel.h"
+#include "fa_plan.h"
+
+using namespace fa;
+
+struct fa_handle_s {
+  fa_desc_t desc{};
+  int device = -1;
+  int num_sms = 0;
+  // plan cache: the per-call arrays the current work list was built from
+  std::vector<int64_t> plan_key;
+  bool plan_valid = false;
+  int32_t n_items = 0;
+  int32_t n_seqs = 0;
+  // device workspace: [error word | pad to 256 B][SeqRec x B][WorkItem x n]
+  void* d_ws = nullptr;
+  size_t ws_bytes = 0;
+  // pinned staging of the work list and the event of its last upload
+  void* h_stage = nullptr;
+  size_t stage_bytes = 0;
+  cudaEvent_t stage_done = nullptr;
+  cudaEvent_t last_call = nullptr;
+  bool any_call = false;
+  // tensor maps of the last call's operands
+  const void* tm_key[3] = {nullptr, nullptr, nullptr};
+  CUtensorMap tm[3];
+  uint64_t timeout_ns = 2000000000ull;
+  uint32_t debug_flags = 0;
+};
+
+namespace {
+
+constexpr size_t kHeaderBytes = 256;
+
+bool env_flag(const char* name) {
+  const char* v = std::getenv(name);
+  return v != nullptr && v[0] != '\0' && v[0] != '0';
+}
+
+fa_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(FA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+fa_status_t bind_device(fa_handle_t h) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (h->device >= 0) {
+    if (dev != h->device)
+      return fail(FA_ERR_PARAM_INVALID, "handle is bound to device %d, current device is %d",
+                  h->device, dev);
+    return FA_OK;
+  }
+  cudaDeviceProp prop;
+  e = cudaGetDeviceProperties(&prop, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(FA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library runs on sm_100 (B200)", dev,
+                prop.major, prop.minor);
+  e = cudaEventCreateWithFlags(&h->stage_done, cudaEventDisableTiming);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreate");
+  e = cudaEventCreateWithFlags(&h->last_call, cudaEventDisableTiming);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreate");
+  h->device = dev;
+  h->num_sms = prop.multiProcessorCount;
+  return FA_OK;
+}
+
+// Make sure the device workspace holds `bytes`; the error word is zeroed
+// whenever the workspace is (re)allocated.
+fa_status_t ensure_workspace(fa_handle_t h, size_t bytes) {
+  if (h->d_ws != nullptr && h->ws_bytes >= bytes) return FA_OK;
+  if (env_flag("FA_TEST_FAIL_ALLOC")) return fail(FA_ERR_ALLOC, "device workspace (test hook)");
+  if (h->d_ws != nullptr) {
+    if (h->any_call) cudaEventSynchronize(h->last_call);
+    cudaFree(h->d_ws);
+    h->d_ws = nullptr;
+    h->ws_bytes = 0;
+  }
+  size_t want = align_up(bytes < 4096 ? 4096 : bytes, 4096);
+  cudaError_t e = cudaMalloc(&h->d_ws, want);
+  if (e != cudaSuccess) {
+    h->d_ws = nullptr;
+    return fail(FA_ERR_ALLOC, "cudaMalloc(%zu): %s", want, cudaGetErrorString(e));
+  }
+  e = cudaMemset(h->d_ws, 0, kHeaderBytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemset");
+  h->ws_bytes = want;
+  return FA_OK;
+}
+
+fa_status_t ensure_stage(fa_handle_t h, size_t bytes) {
+  if (h->h_stage != nullptr && h->stage_bytes >= bytes) return FA_OK;
+  if (h->h_stage != nullptr) {
+    cudaEventSynchronize(h->stage_done);
+    cudaFreeHost(h->h_stage);
+    h->h_stage = nullptr;
+    h->stage_bytes = 0;
+  }
+  size_t want = align_up(bytes < 4096 ? 4096 : bytes, 4096);
+  cudaError_t e = cudaMallocHost(&h->h_stage, want);
+  if (e != cudaSuccess) {
+    h->h_stage = nullptr;
+    return fail(FA_ERR_ALLOC, "cudaMallocHost(%zu): %s", want, cudaGetErrorString(e));
+  }
+  h->stage_bytes = want;
+  return FA_OK;
+}
+
+std::vector<int64_t> make_key(const fa_desc_t* d, const int64_t* prefix, const int64_t* cu_q,
+                              const int64_t* cu_kv, int has_mask) {
+  std::vector<int64_t> key;
+  key.push_back(has_mask);
+  if (d->sparse_mode == 5 || d->sparse_mode == 6) key.insert(key.end(), prefix, prefix + d->B);
+  if (d->layout == FA_TND) {
+    key.insert(key.end(), cu_q, cu_q + d->B);
+    key.insert(key.end(), cu_kv, cu_kv + d->B);
+  }
+  return key;
+}
+
+fa_status_t refresh_plan(fa_handle_t h, const int64_t* prefix, const int64_t* cu_q,
+                         const int64_t* cu_kv, int has_mask, cudaStream_t stream) {
+  std::vector<int64_t> key = make_key(&h->desc, prefix, cu_q, cu_kv, has_mask);
+  if (h->plan_valid && key == h->plan_key) return FA_OK;
+  std::vector<SeqRec> recs = decode_geometry(&h->desc, prefix, cu_q, cu_kv, has_mask);
+  std::vector<WorkItem> items = build_items(&h->desc, recs);
+  if (items.size() > (size_t)0x7fffffff) return fail(FA_ERR_UNSUPPORTED, "too many work items");
+  const size_t seq_bytes = recs.size() * sizeof(SeqRec);
+  const size_t item_bytes = items.size() * sizeof(WorkItem);
+  const size_t payload = align_up(seq_bytes, 256) + item_bytes;
+  fa_status_t st = ensure_workspace(h, kHeaderBytes + payload);
+  if (st != FA_OK) return st;
+  st = ensure_stage(h, payload);
+  if (st != FA_OK) return st;
+  cudaError_t e = cudaEventSynchronize(h->stage_done);  // previous upload has left staging
+  if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+  if (h->any_call) {  // a kernel of this handle on another stream may still read the old list
+    e = cudaStreamWaitEvent(stream, h->last_call, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+  }
+  uint8_t* hs = static_cast<uint8_t*>(h->h_stage);
+  std::memcpy(hs, recs.data(), seq_bytes);
+  if (item_bytes) std::memcpy(hs + align_up(seq_bytes, 256), items.data(), item_bytes);
+  e = cudaMemcpyAsync(static_cast<uint8_t*>(h->d_ws) + kHeaderBytes, hs, payload,
+                      cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(work list)");
+  e = cudaEventRecord(h->stage_done, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  h->plan_key.swap(key);
+  h->plan_valid = true;
+  h->n_items = (int32_t)items.size();
+  h->n_seqs = (int32_t)recs.size();
+  return FA_OK;
+}
+
+// Element strides (batch, head, token) of Q/O or K/V in the handle's layout.
+void operand_strides(const fa_desc_t* d, int64_t S, int64_t* sb, int64_t* sh, int64_t* st) {
+  const int64_t N = d->N, D = d->D;
+  switch (d->layout) {
+    case FA_BNSD:
+      *sb = N * S * D;
+      *sh = S * D;
+      *st = D;
+      break;
+    case FA_BSND:
+      *sb = S * N * D;
+      *sh = D;
+      *st = N * D;
+      break;
+    default:  // TND: batch stride unused (tokens are global)
+      *sb = 0;
+      *sh = D;
+      *st = N * D;
+      break;
+  }
+}
+
+fa_status_t encode_maps(fa_handle_t h, const void* q, const void* k, const void* v) {
+  const void* ptrs[3] = {q, k, v};
+  const fa_desc_t* d = &h->desc;
+  for (int i = 0; i < 3; ++i) {
+    if (h->tm_key[i] == ptrs[i]) continue;
+    const int64_t S = (i == 0) ? d->Sq : d->Skv;
+    int64_t sb, sh, st;
+    operand_strides(d, S, &sb, &sh, &st);
+    const bool tnd = d->layout == FA_TND;
+    // dims (D, S, N, B); TND: (D, T, N, 1) with a dummy (valid) batch stride
+    const int64_t b_extent = tnd ? 1 : d->B;
+    const int64_t b_stride = tnd ? (S > 0 ? S : 1) * d->N * d->D : sb;
+    if (!encode_operand_map(&h->tm[i], ptrs[i], d->D, S, d->N, b_extent, st, sh, b_stride)) {
+      h->tm_key[i] = nullptr;
+      return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed for operand %d", i);
+    }
+    h->tm_key[i] = ptrs[i];
+  }
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status_t fa_create(const fa_desc_t* desc, fa_handle_t* out) {
+  clear_error();
+  if (!out) return fail(FA_ERR_NULLPTR, "out is NULL");
+  *out = nullptr;
+  fa_status_t st = validate_desc(desc);
+  if (st != FA_OK) return st;
+  if (env_flag("FA_TEST_FAIL_ALLOC")) return fail(FA_ERR_ALLOC, "handle (test hook)");
+  fa_handle_t h = new (std::nothrow) fa_handle_s();
+  if (!h) return fail(FA_ERR_ALLOC, "handle");
+  h->desc = *desc;
+  if (const char* t = std::getenv("FA_WAIT_TIMEOUT_MS")) {
+    long long ms = std::atoll(t);
+    if (ms > 0) h->timeout_ns = (uint64_t)ms * 1000000ull;
+  }
+  if (env_flag("FA_TEST_DROP_FIRST_Q")) h->debug_flags |= kDebugDropFirstQ;
+  *out = h;
+  return FA_OK;
+}
+
+fa_status_t fa_fwd(fa_handle_t h, const void* q, const void* k, const void* v,
+                   const uint8_t* atten_mask, const int64_t* prefix,
+                   const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen, void* o,
+                   float* lse, void* cuda_stream) {
+  clear_error();
+  if (!h) return fail(FA_ERR_NULLPTR, "handle is NULL");
+  if (!q || !k || !v || !o || !lse) return fail(FA_ERR_NULLPTR, "q, k, v, o and lse are required");
+  const fa_desc_t* d = &h->desc;
+  const int m = d->sparse_mode;
+  const int has_mask = (m <= 1) && atten_mask != nullptr;
+  fa_status_t st = validate_call(d, prefix, actual_seq_qlen, actual_seq_kvlen, has_mask);
+  if (st != FA_OK) return st;
+  const uintptr_t align = (uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)o;
+  if (align & 15u) return fail(FA_ERR_PARAM_INVALID, "q, k, v and o must be 16-byte aligned");
+  if ((uintptr_t)lse & 3u) return fail(FA_ERR_PARAM_INVALID, "lse must be 4-byte aligned");
+  st = bind_device(h);
+  if (st != FA_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  st = refresh_plan(h, prefix, actual_seq_qlen, actual_seq_kvlen, has_mask, stream);
+  if (st != FA_OK) return st;
+  if (h->n_items == 0) return FA_OK;  // no query rows: nothing to write
+  st = encode_maps(h, q, k, v);
+  if (st != FA_OK) return st;
+
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.tm_q = h->tm[0];
+  p.tm_k = h->tm[1];
+  p.tm_v = h->tm[2];
+  uint8_t* ws = static_cast<uint8_t*>(h->d_ws);
+  p.err_word = reinterpret_cast<unsigned int*>(ws);
+  p.seqs = reinterpret_cast<const SeqRec*>(ws + kHeaderBytes);
+  p.items = reinterpret_cast<const WorkItem*>(
+      ws + kHeaderBytes + align_up((size_t)h->n_seqs * sizeof(SeqRec), 256));
+  p.o = o;
+  p.lse = lse;
+  p.mask = atten_mask;
+  operand_strides(d, d->Sq, &p.o_sb, &p.o_sh, &p.o_st);
+  if (d->layout == FA_TND) {
+    p.l_sb = 0;
+    p.l_sh = d->Sq;
+  } else {
+    p.l_sb = d->N * d->Sq;
+    p.l_sh = d->Sq;
+  }
+  if (has_mask) {
+    const int64_t plane = d->Sq * d->Skv;
+    p.m_si = d->Skv;
+    p.m_sb = (d->mask_kind == FA_MASK_SS) ? 0 : (d->mask_kind == FA_MASK_B1SS ? plane : d->N * plane);
+    p.m_sh = (d->mask_kind == FA_MASK_BNSS) ? plane : 0;
+  }
+  p.n_items = h->n_items;
+  p.tnd = d->layout == FA_TND ? 1 : 0;
+  p.scale_log2 = (float)(d->scale * 1.4426950408889634073599);
+  p.debug_flags = h->debug_flags;
+  p.timeout_ns = h->timeout_ns;
+  const int grid = h->n_items < h->num_sms ? h->n_items : h->num_sms;
+  const char* why = nullptr;
+  cudaError_t e = launch_fwd((int)d->D, p, grid, stream, &why);
+  if (e != cudaSuccess) {
+    if (why) return fail(FA_ERR_UNSUPPORTED, "launch refused: %s", why);
+    return cuda_fail(e, "kernel launch");
+  }
+  e = cudaEventRecord(h->last_call, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  h->any_call = true;
+  return FA_OK;
+}
+
+fa_status_t fa_sync_status(fa_handle_t h) {
+  clear_error();
+  if (!h) return fail(FA_ERR_NULLPTR, "handle is NULL");
+  if (!h->any_call) return FA_OK;
+  cudaError_t e = cudaEventSynchronize(h->last_call);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+  unsigned int word = 0;
+  e = cudaMemcpy(&word, h->d_ws, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(error word)");
+  if (word == 0) return FA_OK;
+  e = cudaMemset(h->d_ws, 0, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(error word)");
+  if (word & kErrTimeout)
+    return fail(FA_ERR_TIMEOUT, "a device-side wait gave up (site %u); outputs are undefined",
+                (word >> kErrWhereShift) & 0xffu);
+  return fail(FA_ERR_DEVICE, "device error word 0x%08x", word);
+}
+
+fa_status_t fa_destroy(fa_handle_t h) {
+  clear_error();
+  if (!h) return FA_OK;
+  if (h->any_call) cudaEventSynchronize(h->last_call);
+  if (h->stage_done) cudaEventSynchronize(h->stage_done);
+  if (h->d_ws) cudaFree(h->d_ws);
+  if (h->h_stage) cudaFreeHost(h->h_stage);
+  if (h->stage_done) cudaEventDestroy(h->stage_done);
+  if (h->last_call) cudaEventDestroy(h->last_call);
+  delete h;
+  return FA_OK;
+}
+
+}  // extern "C"

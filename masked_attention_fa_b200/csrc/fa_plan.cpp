@@ -1,0 +1,371 @@
+// Host side of the C ABI that needs no device: argument validation, the
+// per-sequence geometry decode and the tile scheduler's work list.
+//
+// Validation rules come from the Ascend CANN page "sparseMode参数说明":
+//   sparseMode=0 (the two 说明 notes on negative nextTokens / preTokens),
+//   sparseMode=4 (pre and next must intersect),
+//   sparseMode=7 and sparseMode=8 (the band-piece conditions and Sq <= Skv
+//   for the other batches).
+#include "fa_plan.h"
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+namespace fa {
+
+static thread_local std::string g_last_error;
+
+fa_status_t fail(fa_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+void clear_error() { g_last_error.clear(); }
+const char* last_error() { return g_last_error.c_str(); }
+
+static int64_t clamp_off(__int128 x) {
+  if (x < -(__int128)kUnbounded) return -kUnbounded;
+  if (x > (__int128)kUnbounded) return kUnbounded;
+  return (int64_t)x;
+}
+
+fa_status_t validate_desc(const fa_desc_t* d) {
+  if (!d) return fail(FA_ERR_NULLPTR, "desc is NULL");
+  if (d->layout < FA_BNSD || d->layout > FA_TND)
+    return fail(FA_ERR_PARAM_INVALID, "layout %d is not BNSD(0), BSND(1) or TND(2)", d->layout);
+  if (d->sparse_mode < 0 || d->sparse_mode > 8)
+    return fail(FA_ERR_PARAM_INVALID, "sparse_mode %d is outside 0..8", d->sparse_mode);
+  if (d->reserved != 0) return fail(FA_ERR_PARAM_INVALID, "reserved field must be 0");
+  if (d->B < 1 || d->N < 1 || d->D < 1)
+    return fail(FA_ERR_SHAPE, "B, N and D must be >= 1 (got %lld, %lld, %lld)", (long long)d->B,
+                (long long)d->N, (long long)d->D);
+  if (d->Sq < 0 || d->Skv < 0)
+    return fail(FA_ERR_SHAPE, "Sq and Skv must be >= 0 (got %lld, %lld)", (long long)d->Sq,
+                (long long)d->Skv);
+  if (d->Sq >= kUnbounded || d->Skv >= kUnbounded || d->B >= kUnbounded || d->N >= 65536)
+    return fail(FA_ERR_UNSUPPORTED, "sizes too large (Sq, Skv, B < 2^30, N < 65536)");
+  if (d->D != 64 && d->D != 128)
+    return fail(FA_ERR_UNSUPPORTED, "head dim D=%lld: this build supports D in {64, 128}",
+                (long long)d->D);
+  // Element counts of the largest operand must stay well inside TMA's
+  // 2^40-byte stride range.
+  const __int128 rows_q = (d->layout == FA_TND) ? (__int128)d->Sq : (__int128)d->B * d->Sq;
+  const __int128 rows_kv = (d->layout == FA_TND) ? (__int128)d->Skv : (__int128)d->B * d->Skv;
+  if (std::max(rows_q, rows_kv) * d->N * d->D * 2 >= ((__int128)1 << 39))
+    return fail(FA_ERR_UNSUPPORTED, "operands larger than 2^39 bytes");
+  if (!(d->scale > 0.0) || !std::isfinite(d->scale))
+    return fail(FA_ERR_PARAM_INVALID, "scale must be finite and > 0 (got %g)", d->scale);
+  if (d->mask_kind < FA_MASK_NONE || d->mask_kind > FA_MASK_BNSS)
+    return fail(FA_ERR_PARAM_INVALID, "mask_kind %d is not NONE/SS/B1SS/BNSS", d->mask_kind);
+  const int m = d->sparse_mode;
+  if (m >= 2 && d->mask_kind != FA_MASK_NONE)
+    return fail(FA_ERR_PARAM_INVALID,
+                "sparse_mode %d derives its mask from the geometry; mask_kind must be NONE", m);
+  if (m == 1 && d->mask_kind == FA_MASK_NONE)
+    return fail(FA_ERR_PARAM_INVALID, "sparse_mode 1 (allMask) needs a mask_kind");
+  if (d->layout == FA_TND && d->mask_kind != FA_MASK_NONE)
+    return fail(FA_ERR_UNSUPPORTED, "an attenMask with the TND layout is not supported");
+  if ((m == 7 || m == 8) && d->layout != FA_TND)
+    return fail(FA_ERR_PARAM_INVALID, "sparse_mode %d is a varlen mode and needs layout TND", m);
+  if (m == 0 && d->mask_kind != FA_MASK_NONE) {
+    const int64_t pre = d->pre_tokens, nxt = d->next_tokens;
+    if (nxt < 0) {
+      if ((__int128)pre < -(__int128)nxt)
+        return fail(FA_ERR_PARAM_INVALID,
+                    "sparse_mode 0: next_tokens < 0 needs pre_tokens >= |next_tokens|");
+      if (-(__int128)nxt >= d->Skv)
+        return fail(FA_ERR_PARAM_INVALID, "sparse_mode 0: |next_tokens| must be < Skv");
+    }
+    if (pre < 0) {
+      if ((__int128)nxt < -(__int128)pre)
+        return fail(FA_ERR_PARAM_INVALID,
+                    "sparse_mode 0: pre_tokens < 0 needs next_tokens >= |pre_tokens|");
+      if (-(__int128)pre >= d->Sq)
+        return fail(FA_ERR_PARAM_INVALID, "sparse_mode 0: |pre_tokens| must be < Sq");
+    }
+  }
+  if (m == 4 && (__int128)d->pre_tokens + (__int128)d->next_tokens < 0)
+    return fail(FA_ERR_PARAM_INVALID,
+                "sparse_mode 4: the pre/next band must intersect (pre_tokens + next_tokens >= 0)");
+  return FA_OK;
+}
+
+static void seq_extent(const fa_desc_t* d, const int64_t* cu_q, const int64_t* cu_kv, int64_t b,
+                       int64_t* q_off, int64_t* kv_off, int64_t* sq, int64_t* skv) {
+  if (d->layout == FA_TND) {
+    *q_off = b == 0 ? 0 : cu_q[b - 1];
+    *kv_off = b == 0 ? 0 : cu_kv[b - 1];
+    *sq = cu_q[b] - *q_off;
+    *skv = cu_kv[b] - *kv_off;
+  } else {
+    *q_off = *kv_off = 0;
+    *sq = d->Sq;
+    *skv = d->Skv;
+  }
+}
+
+fa_status_t validate_call(const fa_desc_t* d, const int64_t* prefix, const int64_t* cu_q,
+                          const int64_t* cu_kv, int has_mask) {
+  fa_status_t st = validate_desc(d);
+  if (st != FA_OK) return st;
+  const int m = d->sparse_mode;
+  if (m == 1 && !has_mask) return fail(FA_ERR_NULLPTR, "sparse_mode 1 (allMask) needs atten_mask");
+  if (m == 0 && has_mask && d->mask_kind == FA_MASK_NONE)
+    return fail(FA_ERR_PARAM_INVALID, "atten_mask given but mask_kind is NONE");
+  if (d->layout == FA_TND) {
+    if (!cu_q || !cu_kv)
+      return fail(FA_ERR_NULLPTR, "TND needs actual_seq_qlen and actual_seq_kvlen");
+    int64_t pq = 0, pk = 0;
+    for (int64_t b = 0; b < d->B; ++b) {
+      if (cu_q[b] < pq || cu_kv[b] < pk)
+        return fail(FA_ERR_SHAPE, "actual_seq lengths must be non-decreasing cumulative ends "
+                    "(entry %lld)", (long long)b);
+      pq = cu_q[b];
+      pk = cu_kv[b];
+    }
+    if (pq != d->Sq || pk != d->Skv)
+      return fail(FA_ERR_SHAPE,
+                  "last actual_seq_qlen/kvlen (%lld, %lld) must equal Sq/Skv (%lld, %lld)",
+                  (long long)pq, (long long)pk, (long long)d->Sq, (long long)d->Skv);
+  }
+  if (m == 5 || m == 6) {
+    if (!prefix) return fail(FA_ERR_NULLPTR, "sparse_mode %d needs the prefix array", m);
+    for (int64_t b = 0; b < d->B; ++b) {
+      int64_t qo, ko, sq, skv;
+      seq_extent(d, cu_q, cu_kv, b, &qo, &ko, &sq, &skv);
+      if (prefix[b] < 0 || prefix[b] > skv)
+        return fail(FA_ERR_PARAM_INVALID, "prefix[%lld]=%lld must be in [0, Skv_b=%lld]",
+                    (long long)b, (long long)prefix[b], (long long)skv);
+    }
+  }
+  if (m == 7 || m == 8) {
+    int64_t band = -1;
+    for (int64_t i = 0; i < d->B; ++i) {
+      int64_t b = (m == 7) ? d->B - 1 - i : i;
+      int64_t qo, ko, sq, skv;
+      seq_extent(d, cu_q, cu_kv, b, &qo, &ko, &sq, &skv);
+      if (sq > 0) {
+        band = b;
+        break;
+      }
+    }
+    if (band >= 0) {
+      int64_t qo, ko, sq, skv;
+      seq_extent(d, cu_q, cu_kv, band, &qo, &ko, &sq, &skv);
+      const __int128 pre = d->pre_tokens, nxt = d->next_tokens;
+      if (pre < skv)
+        return fail(FA_ERR_PARAM_INVALID,
+                    "sparse_mode %d: pre_tokens (%lld) must be >= Skv of the band sequence (%lld)",
+                    m, (long long)d->pre_tokens, (long long)skv);
+      if (m == 7 && (nxt > 0 || nxt < (__int128)(sq - skv)))
+        return fail(FA_ERR_PARAM_INVALID,
+                    "sparse_mode 7: need last_Sq - last_Skv (%lld) <= next_tokens (%lld) <= 0",
+                    (long long)(sq - skv), (long long)d->next_tokens);
+      if (m == 8 && nxt < (__int128)(sq - skv))
+        return fail(FA_ERR_PARAM_INVALID,
+                    "sparse_mode 8: need next_tokens (%lld) >= first_Sq - first_Skv (%lld)",
+                    (long long)d->next_tokens, (long long)(sq - skv));
+      if (m == 7) {
+        for (int64_t b = 0; b < d->B; ++b) {
+          if (b == band) continue;
+          seq_extent(d, cu_q, cu_kv, b, &qo, &ko, &sq, &skv);
+          if (sq > skv)
+            return fail(FA_ERR_PARAM_INVALID,
+                        "sparse_mode 7: non-band sequence %lld has Sq (%lld) > Skv (%lld)",
+                        (long long)b, (long long)sq, (long long)skv);
+        }
+      }
+    }
+  }
+  return FA_OK;
+}
+
+// Rows of sequence b see keys [max(0, i + lo), min(Skv-1, max(i + hi, prefix-1))].
+std::vector<SeqRec> decode_geometry(const fa_desc_t* d, const int64_t* prefix,
+                                    const int64_t* cu_q, const int64_t* cu_kv, int has_mask) {
+  const int m = d->sparse_mode;
+  const bool dense = (m == 1) || (m == 0 && has_mask);
+  int64_t first_ne = -1, last_ne = -1;
+  for (int64_t b = 0; b < d->B; ++b) {
+    int64_t qo, ko, sq, skv;
+    seq_extent(d, cu_q, cu_kv, b, &qo, &ko, &sq, &skv);
+    if (sq > 0) {
+      if (first_ne < 0) first_ne = b;
+      last_ne = b;
+    }
+  }
+  std::vector<SeqRec> recs((size_t)d->B);
+  for (int64_t b = 0; b < d->B; ++b) {
+    int64_t qo, ko, sq, skv;
+    seq_extent(d, cu_q, cu_kv, b, &qo, &ko, &sq, &skv);
+    const __int128 delta = (__int128)skv - sq;
+    int64_t lo = -kUnbounded, hi = kUnbounded, pfx = 0;
+    int rule = m;
+    if (m == 7) rule = (b == last_ne) ? 4 : 3;
+    if (m == 8) rule = (b == first_ne) ? 4 : 2;
+    switch (rule) {
+      case 0:
+        if (has_mask) {  // band from the top-left, inclusive bounds
+          lo = clamp_off(-(__int128)d->pre_tokens);
+          hi = clamp_off((__int128)d->next_tokens);
+        }
+        break;
+      case 1:
+        break;
+      case 2:  // leftUpCausal
+        hi = 0;
+        break;
+      case 3:  // rightDownCausal
+        hi = clamp_off(delta);
+        break;
+      case 4:  // band from the bottom-right
+        lo = clamp_off(delta - d->pre_tokens);
+        hi = clamp_off(delta + d->next_tokens);
+        break;
+      case 5:
+      case 6:  // rightDownCausal plus prefix[b] leading columns
+        hi = clamp_off(delta);
+        pfx = prefix[b];
+        break;
+    }
+    SeqRec& r = recs[(size_t)b];
+    r.q_off = (int32_t)qo;
+    r.kv_off = (int32_t)ko;
+    r.sq = (int32_t)sq;
+    r.skv = (int32_t)skv;
+    r.lo_off = (int32_t)lo;
+    r.hi_off = (int32_t)hi;
+    r.prefix = (int32_t)pfx;
+    r.flags = dense ? kSeqDenseMask : 0;
+  }
+  return recs;
+}
+
+static int32_t tiles_of(const TileRange& t) { return t.hi > t.lo ? t.hi - t.lo : 0; }
+
+// One item per (sequence, head, 256-row block). Items are sorted by
+// descending cost (longest-processing-time first), ties in index order.
+std::vector<WorkItem> build_items(const fa_desc_t* d, const std::vector<SeqRec>& recs) {
+  std::vector<WorkItem> items;
+  for (int64_t b = 0; b < d->B; ++b) {
+    const SeqRec& s = recs[(size_t)b];
+    if (s.sq <= 0) continue;
+    const int32_t nblk = (s.sq + kBlockM - 1) / kBlockM;
+    for (int32_t qb = 0; qb < nblk; ++qb) {
+      int32_t cost = 0;
+      for (int st = 0; st < kSubTiles; ++st)
+        cost += tiles_of(tile_range(s, (int64_t)qb * kBlockM + st * kTileM));
+      for (int64_t h = 0; h < d->N; ++h)
+        items.push_back(WorkItem{(int32_t)b, (int32_t)h, qb, cost});
+    }
+  }
+  std::stable_sort(items.begin(), items.end(),
+                   [](const WorkItem& a, const WorkItem& c) { return a.cost > c.cost; });
+  return items;
+}
+
+int64_t visible_pairs(const fa_desc_t* d, const std::vector<SeqRec>& recs) {
+  int64_t total = 0;
+  for (const SeqRec& s : recs) {
+    int64_t per_head = 0;
+    for (int64_t i = 0; i < s.sq; ++i) {
+      int64_t jlo = imax64(0, row_lo(s, i));
+      int64_t jhi = imin64((int64_t)s.skv - 1, row_hi(s, i));
+      if (jhi >= jlo) per_head += jhi - jlo + 1;
+    }
+    total += per_head * d->N;
+  }
+  return total;
+}
+
+int32_t tile_class(const SeqRec& s, int64_t qt, int64_t kt) {
+  const int64_t r0 = qt * kTileM;
+  if (r0 >= s.sq || kt < 0 || kt * kTileN >= s.skv) return FA_TILE_EMPTY;
+  const TileRange t = tile_range(s, r0);
+  if (kt < t.lo || kt >= t.hi) return FA_TILE_EMPTY;
+  if (kt >= t.full_lo && kt < t.full_hi) return FA_TILE_FULL;
+  return FA_TILE_PARTIAL;
+}
+
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_last_error(void) { return last_error(); }
+
+int32_t fa_version(void) { return FA_VERSION; }
+
+fa_status_t fa_validate(const fa_desc_t* desc, const int64_t* prefix,
+                        const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
+                        int32_t has_mask) {
+  clear_error();
+  return validate_call(desc, prefix, actual_seq_qlen, actual_seq_kvlen, has_mask);
+}
+
+fa_status_t fa_visible_pairs(const fa_desc_t* desc, const int64_t* prefix,
+                             const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
+                             int32_t has_mask, int64_t* pairs_out) {
+  clear_error();
+  if (!pairs_out) return fail(FA_ERR_NULLPTR, "pairs_out is NULL");
+  fa_status_t st = validate_call(desc, prefix, actual_seq_qlen, actual_seq_kvlen, has_mask);
+  if (st != FA_OK) return st;
+  if (desc->sparse_mode == 1 || (desc->sparse_mode == 0 && has_mask))
+    return fail(FA_ERR_UNSUPPORTED, "visible pairs of a dense-mask call depend on the mask data");
+  auto recs = decode_geometry(desc, prefix, actual_seq_qlen, actual_seq_kvlen, has_mask);
+  *pairs_out = visible_pairs(desc, recs);
+  return FA_OK;
+}
+
+int32_t fa_tile_class(const fa_desc_t* desc, const int64_t* prefix,
+                      const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
+                      int32_t has_mask, int64_t b, int64_t qt, int64_t kt) {
+  clear_error();
+  if (validate_call(desc, prefix, actual_seq_qlen, actual_seq_kvlen, has_mask) != FA_OK) return -1;
+  if (b < 0 || b >= desc->B || qt < 0) {
+    fail(FA_ERR_PARAM_INVALID, "tile index out of range");
+    return -1;
+  }
+  auto recs = decode_geometry(desc, prefix, actual_seq_qlen, actual_seq_kvlen, has_mask);
+  return tile_class(recs[(size_t)b], qt, kt);
+}
+
+fa_status_t fa_plan_stats(const fa_desc_t* desc, const int64_t* prefix,
+                          const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
+                          int32_t has_mask, int64_t* out) {
+  clear_error();
+  if (!out) return fail(FA_ERR_NULLPTR, "out is NULL");
+  fa_status_t st = validate_call(desc, prefix, actual_seq_qlen, actual_seq_kvlen, has_mask);
+  if (st != FA_OK) return st;
+  auto recs = decode_geometry(desc, prefix, actual_seq_qlen, actual_seq_kvlen, has_mask);
+  auto items = build_items(desc, recs);
+  int64_t counts[3] = {0, 0, 0};
+  for (const SeqRec& s : recs) {
+    const int64_t nqt = (s.sq + kTileM - 1) / kTileM;
+    const int64_t nkt = (s.skv + kTileN - 1) / kTileN;
+    for (int64_t qt = 0; qt < nqt; ++qt) {
+      const TileRange t = tile_range(s, qt * kTileM);
+      const int64_t nonempty = t.hi - t.lo;
+      const int64_t full = t.full_hi - t.full_lo;
+      counts[FA_TILE_FULL] += full * desc->N;
+      counts[FA_TILE_PARTIAL] += (nonempty - full) * desc->N;
+      counts[FA_TILE_EMPTY] += (nkt - nonempty) * desc->N;
+    }
+  }
+  out[0] = (int64_t)items.size();
+  out[1] = counts[FA_TILE_EMPTY];
+  out[2] = counts[FA_TILE_PARTIAL];
+  out[3] = counts[FA_TILE_FULL];
+  return FA_OK;
+}
+
+}  // extern "C"

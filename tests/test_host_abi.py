@@ -1,0 +1,268 @@
+"""Host-side checks of the C-ABI library (no GPU needed, no device work).
+
+- the library loads and exports every entry point include/fa.h declares;
+- validation returns the documented status for each constraint of the
+  Ascend "sparseMode参数说明" page (sparseMode=0 notes, =4, =7, =8);
+- the scheduler's visible-pair count and tile classes agree with the fp64
+  oracle's explicit masks.
+"""
+import os
+import re
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+import masked_attention_fa_b200 as fa
+import oracle
+from oracle import Problem
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from masked_attention_fa_b200 import build
+    build.build()
+
+
+def test_library_exports_every_declared_entry_point():
+    with open(os.path.join(ROOT, "include", "fa.h")) as f:
+        header = f.read()
+    declared = set(re.findall(r"^\s*(?:fa_status_t|int32_t|const char\*)\s+(fa_\w+)\s*\(",
+                              header, re.M))
+    assert declared >= {"fa_create", "fa_fwd", "fa_destroy", "fa_last_error"}
+    lib = fa.load_library()
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(fa.EXPORTED) == declared
+    assert fa.fa_version() == 1
+
+
+def _status(**kw):
+    arrays = {k: kw.pop(k) for k in ("prefix", "actual_seq_qlen", "actual_seq_kvlen", "has_mask")
+              if k in kw}
+    return fa.STATUS[fa.fa_validate(fa.make_desc(**kw), **arrays)]
+
+
+BASE = dict(layout="BNSD", B=1, N=2, Sq=64, Skv=64, D=128)
+
+
+def test_valid_descriptors():
+    assert _status(**BASE, sparse_mode=2) == "FA_OK"
+    assert _status(**BASE, sparse_mode=0) == "FA_OK"
+    assert _status(**dict(BASE, D=64), sparse_mode=3) == "FA_OK"
+    assert _status(**BASE, sparse_mode=4, pre_tokens=2147483647, next_tokens=2147483647) == "FA_OK"
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(layout=7), "FA_ERR_PARAM_INVALID"),
+    (dict(sparse_mode=9), "FA_ERR_PARAM_INVALID"),
+    (dict(B=0), "FA_ERR_SHAPE"),
+    (dict(Sq=-1), "FA_ERR_SHAPE"),
+    (dict(D=96), "FA_ERR_UNSUPPORTED"),
+    (dict(D=256), "FA_ERR_UNSUPPORTED"),
+    (dict(scale=0.0), "FA_ERR_PARAM_INVALID"),
+    (dict(scale=float("nan")), "FA_ERR_PARAM_INVALID"),
+    (dict(sparse_mode=2, mask_kind="SS"), "FA_ERR_PARAM_INVALID"),
+    (dict(sparse_mode=1), "FA_ERR_PARAM_INVALID"),
+    (dict(sparse_mode=7), "FA_ERR_PARAM_INVALID"),
+])
+def test_descriptor_errors(kw, status):
+    args = dict(BASE)
+    args.update(kw)
+    args.setdefault("sparse_mode", 0)
+    assert _status(**args) == status
+
+
+def test_mode0_negative_pre_next_constraints():
+    """sparseMode=0 notes: next < 0 needs pre >= |next| and |next| < Skv;
+    pre < 0 needs next >= |pre| and |pre| < Sq (only when a mask is given)."""
+    m = dict(BASE, sparse_mode=0, mask_kind="SS", has_mask=True)
+    assert _status(**m, pre_tokens=9, next_tokens=-3) == "FA_OK"
+    assert _status(**m, pre_tokens=3, next_tokens=-3) == "FA_OK"
+    assert _status(**m, pre_tokens=2, next_tokens=-3) == "FA_ERR_PARAM_INVALID"
+    assert _status(**m, pre_tokens=100, next_tokens=-64) == "FA_ERR_PARAM_INVALID"
+    assert _status(**m, pre_tokens=-3, next_tokens=7) == "FA_OK"
+    assert _status(**m, pre_tokens=-3, next_tokens=2) == "FA_ERR_PARAM_INVALID"
+    assert _status(**m, pre_tokens=-64, next_tokens=100) == "FA_ERR_PARAM_INVALID"
+    # without a mask pre/next are ignored
+    assert _status(**BASE, sparse_mode=0, pre_tokens=2, next_tokens=-3) == "FA_OK"
+    # a mask pointer with mask_kind NONE cannot be interpreted
+    assert _status(**BASE, sparse_mode=0, has_mask=True) == "FA_ERR_PARAM_INVALID"
+    assert _status(**dict(BASE, mask_kind="SS"), sparse_mode=1) == "FA_ERR_NULLPTR"
+
+
+def test_mode4_band_must_intersect():
+    assert _status(**BASE, sparse_mode=4, pre_tokens=3, next_tokens=-3) == "FA_OK"
+    assert _status(**BASE, sparse_mode=4, pre_tokens=3, next_tokens=-4) == "FA_ERR_PARAM_INVALID"
+
+
+def test_prefix_and_varlen_arrays():
+    assert _status(**BASE, sparse_mode=5) == "FA_ERR_NULLPTR"
+    assert _status(**BASE, sparse_mode=5, prefix=[65]) == "FA_ERR_PARAM_INVALID"
+    assert _status(**BASE, sparse_mode=6, prefix=[64]) == "FA_OK"
+    t = dict(layout="TND", B=2, N=1, Sq=5, Skv=9, D=64, sparse_mode=3)
+    assert _status(**t) == "FA_ERR_NULLPTR"
+    assert _status(**t, actual_seq_qlen=[3, 5], actual_seq_kvlen=[3, 9]) == "FA_OK"
+    assert _status(**t, actual_seq_qlen=[3, 4], actual_seq_kvlen=[3, 9]) == "FA_ERR_SHAPE"
+    assert _status(**t, actual_seq_qlen=[6, 5], actual_seq_kvlen=[3, 9]) == "FA_ERR_SHAPE"
+    assert _status(**dict(t, mask_kind="SS", sparse_mode=0)) == "FA_ERR_UNSUPPORTED"
+
+
+def test_mode7_mode8_worked_examples_validate():
+    """The two cards of each worked split on the sparseMode page validate,
+    and breaking each listed condition is rejected."""
+    c7 = dict(layout="TND", B=2, N=1, Sq=5, Skv=9, D=64, sparse_mode=7)
+    arr7 = dict(actual_seq_qlen=[3, 5], actual_seq_kvlen=[3, 9])
+    assert _status(**c7, pre_tokens=6, next_tokens=-2, **arr7) == "FA_OK"
+    assert _status(**c7, pre_tokens=5, next_tokens=-2, **arr7) == "FA_ERR_PARAM_INVALID"
+    assert _status(**c7, pre_tokens=6, next_tokens=1, **arr7) == "FA_ERR_PARAM_INVALID"
+    assert _status(**c7, pre_tokens=6, next_tokens=-5, **arr7) == "FA_ERR_PARAM_INVALID"
+    # a non-band sequence with Sq > Skv
+    assert _status(**dict(c7, Skv=8), pre_tokens=6, next_tokens=-2, actual_seq_qlen=[3, 5],
+                   actual_seq_kvlen=[2, 8]) == "FA_ERR_PARAM_INVALID"
+    c8 = dict(layout="TND", B=3, N=1, Sq=12, Skv=13, D=64, sparse_mode=8)
+    arr8 = dict(actual_seq_qlen=[3, 8, 12], actual_seq_kvlen=[4, 9, 13])
+    assert _status(**c8, pre_tokens=4, next_tokens=1, **arr8) == "FA_OK"
+    assert _status(**c8, pre_tokens=3, next_tokens=1, **arr8) == "FA_ERR_PARAM_INVALID"
+    assert _status(**c8, pre_tokens=4, next_tokens=-2, **arr8) == "FA_ERR_PARAM_INVALID"
+    assert _status(**dict(c8, layout="BNSD"), pre_tokens=4, next_tokens=1) == "FA_ERR_PARAM_INVALID"
+
+
+def test_create_rejects_and_alloc_injection():
+    with pytest.raises(fa.FaError) as e:
+        fa.fa_create(fa.make_desc("BNSD", 1, 1, 8, 8, 80, 2))
+    assert e.value.name == "FA_ERR_UNSUPPORTED" and "D=80" in str(e.value)
+    h = fa.fa_create(fa.make_desc("BNSD", 1, 1, 8, 8, 64, 2))
+    fa.fa_destroy(h)
+    fa.fa_destroy(None)
+    code = ("import masked_attention_fa_b200 as fa\n"
+            "try:\n    fa.fa_create(fa.make_desc('BNSD',1,1,8,8,64,2))\n"
+            "except fa.FaError as e:\n    print(e.name)\n")
+    env = dict(os.environ, FA_TEST_FAIL_ALLOC="1", PYTHONPATH=ROOT)
+    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                         cwd=ROOT, timeout=120)
+    assert out.stdout.strip() == "FA_ERR_ALLOC", out.stderr
+
+
+# ---------------------------------------------------------------- scheduler vs oracle
+
+def _random_problem(rng, mode):
+    """A small random valid call of `mode` with lengths that cross 128-key tiles."""
+    N = 1
+    if mode in (7, 8):
+        nseq = int(rng.integers(1, 4))
+        lens = []
+        for _ in range(nseq):
+            sq = int(rng.integers(0, 300))
+            skv = sq + int(rng.integers(0, 200))
+            lens.append((sq, skv))
+        nonempty = [i for i, (a, _) in enumerate(lens) if a > 0]
+        if not nonempty:
+            lens[0] = (5, 9)
+            nonempty = [0]
+        band = nonempty[-1] if mode == 7 else nonempty[0]
+        sq, skv = lens[band]
+        pre = skv + int(rng.integers(0, 50))
+        if mode == 7:
+            nxt = int(rng.integers(sq - skv, 1))
+        else:
+            nxt = sq - skv + int(rng.integers(0, 100))
+        cu_q = np.cumsum([a for a, _ in lens]).tolist()
+        cu_k = np.cumsum([b for _, b in lens]).tolist()
+        return dict(layout="TND", B=nseq, N=N, Sq=cu_q[-1], Skv=cu_k[-1], D=64, sparse_mode=mode,
+                    pre_tokens=pre, next_tokens=nxt, actual_seq_qlen=cu_q, actual_seq_kvlen=cu_k)
+    Sq = int(rng.integers(1, 400))
+    Skv = int(rng.integers(1, 400))
+    kw = dict(layout="BNSD", B=2, N=N, Sq=Sq, Skv=Skv, D=64, sparse_mode=mode)
+    if mode == 4:
+        pre = int(rng.integers(-100, 500))
+        kw.update(pre_tokens=pre, next_tokens=int(rng.integers(-pre, 500)))
+    if mode in (5, 6):
+        kw["prefix"] = [int(rng.integers(0, Skv + 1)) for _ in range(2)]
+    return kw
+
+
+def _split(kw):
+    desc_kw = {k: v for k, v in kw.items()
+               if k not in ("prefix", "actual_seq_qlen", "actual_seq_kvlen")}
+    arrays = {k: kw[k] for k in ("prefix", "actual_seq_qlen", "actual_seq_kvlen") if k in kw}
+    return desc_kw, arrays
+
+
+@pytest.mark.parametrize("mode", [0, 2, 3, 4, 5, 6, 7, 8])
+def test_visible_pairs_match_oracle_counts(mode):
+    rng = np.random.default_rng(100 + mode)
+    for _ in range(6):
+        kw = _random_problem(rng, mode)
+        desc_kw, arrays = _split(kw)
+        assert fa.fa_validate(fa.make_desc(**desc_kw), **arrays) == 0, kw
+        got = fa.fa_visible_pairs(fa.make_desc(**desc_kw), **arrays)
+        pb = Problem(**kw)
+        assert got == oracle.visible_count(pb), kw
+
+
+@pytest.mark.parametrize("mode", [0, 2, 3, 4, 5, 6, 7, 8])
+def test_tile_classes_match_oracle_masks(mode):
+    """EMPTY <=> the tile has no visible pair; FULL <=> every stored row sees
+    all 128 keys of the tile; PARTIAL otherwise."""
+    rng = np.random.default_rng(200 + mode)
+    for _ in range(4):
+        kw = _random_problem(rng, mode)
+        desc_kw, arrays = _split(kw)
+        desc = fa.make_desc(**desc_kw)
+        pb = Problem(**kw)
+        for b in range(pb.B):
+            _, _, sq, skv = pb.seq(b)
+            if sq == 0:
+                continue
+            vis = oracle.mask_matrix(pb, b)
+            for qt in range((sq + 127) // 128):
+                for kt in range((skv + 127) // 128 + 1):
+                    blk = vis[qt * 128:(qt + 1) * 128, kt * 128:(kt + 1) * 128]
+                    cls = fa.fa_tile_class(desc, b, qt, kt, **arrays)
+                    if blk.size == 0 or not blk.any():
+                        want = fa.FA_TILE_EMPTY
+                    elif blk.all() and blk.shape[1] == 128:
+                        want = fa.FA_TILE_FULL
+                    else:
+                        want = fa.FA_TILE_PARTIAL
+                    assert cls == want, (kw, b, qt, kt)
+
+
+def test_dense_mask_tiles_are_never_full():
+    S = 300
+    mask = np.zeros((S, S), np.uint8)
+    desc = fa.make_desc("BNSD", 1, 1, S, S, 64, 0, pre_tokens=40, next_tokens=5, mask_kind="SS")
+    pb = Problem("BNSD", 1, 1, S, S, 64, sparse_mode=0, pre_tokens=40, next_tokens=5,
+                 mask=mask, mask_kind="SS")
+    vis = oracle.mask_matrix(pb, 0)
+    for qt in range(3):
+        for kt in range(3):
+            cls = fa.fa_tile_class(desc, 0, qt, kt, has_mask=True)
+            blk = vis[qt * 128:(qt + 1) * 128, kt * 128:(kt + 1) * 128]
+            assert cls != fa.FA_TILE_FULL
+            assert (cls == fa.FA_TILE_EMPTY) == (not blk.any())
+
+
+def test_plan_stats_item_count_and_named_workload_counts():
+    from masked_attention_fa_b200.workloads import named_workloads
+    ws = named_workloads()
+    w = ws["leftup_causal_4k"]
+    d = fa.make_desc(w.layout, w.B, w.N, w.Sq, w.Skv, w.D, w.sparse_mode)
+    items, empty, partial, full = fa.fa_plan_stats(d)
+    assert items == 2 * 16 * 16
+    assert partial == 2 * 16 * 32        # the diagonal tiles
+    assert full == 2 * 16 * (32 * 31 // 2)
+    assert fa.fa_visible_pairs(d) == 268500992
+    w = ws["rightdown_band_2k_8k"]
+    d = fa.make_desc(w.layout, w.B, w.N, w.Sq, w.Skv, w.D, w.sparse_mode, w.pre_tokens,
+                     w.next_tokens)
+    assert fa.fa_visible_pairs(d) == 32 * 2048 * 1025
+    w = ws["prefix_8k"]
+    d = fa.make_desc(w.layout, w.B, w.N, w.Sq, w.Skv, w.D, w.sparse_mode)
+    S = 8192
+    expect = 16 * sum(P * P + S * (S + 1) // 2 - P * (P + 1) // 2 for P in w.prefix)
+    assert fa.fa_visible_pairs(d, prefix=w.prefix) == expect == 2325942272
