@@ -152,6 +152,36 @@ const char* fa_last_error(void);
 /* Library version (FA_VERSION). */
 int32_t fa_version(void);
 
+/*
+ * fa_fwd_noalloc — the same forward as fa_fwd for callers that cannot
+ * allocate memory (for example code running inside a framework that owns
+ * every device allocation through its own pool, a real-time loop that must
+ * not allocate after start-up, or a plugin called from another library's
+ * memory callbacks). The paper has no counterpart of this entry point.
+ *
+ * No handle: the descriptor and all arrays are passed on every call, with
+ * the meaning, layout and validation of fa_create + fa_fwd. The work list
+ * and the error word live in one fixed device array of 1 MiB per device,
+ * held from library load until process exit, instead of a cudaMalloc'd
+ * workspace: the call makes no cudaMalloc, cudaFree or pinned allocation.
+ * Capacity: 256 + 32 * B (rounded up to 256) + 16 * items bytes, where items
+ * = N * sum over sequences of ceil(Sq_b / 256); a problem beyond 1 MiB returns
+ * FA_ERR_UNSUPPORTED before any device work (use fa_create/fa_fwd then).
+ * Sharing: every call shares the array and leaves its work list there; the
+ * error word is cleared at the start of each call. Calls whose kernels
+ * overlap on the GPU race on the array: order them on one stream. Host calls
+ * are serialised internally.
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) and the device's attributes with that device
+ * current; make that first call before any stream capture begins.
+ * A device-side wait that gives up leaves the outputs undefined and is not
+ * reported by this entry point.
+ */
+fa_status_t fa_fwd_noalloc(const fa_desc_t* desc, const void* q, const void* k, const void* v,
+                           const uint8_t* atten_mask, const int64_t* prefix,
+                           const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
+                           void* o, float* lse, void* cuda_stream);
+
 /* ---------------- host-only helpers (no device work) ------------------- */
 
 /*

@@ -89,12 +89,15 @@ def load_library():
     lib.fa_tile_class.restype = ctypes.c_int32
     lib.fa_plan_stats.argtypes = [dp, i64p, i64p, i64p, ctypes.c_int32, i64p]
     lib.fa_plan_stats.restype = st
+    lib.fa_fwd_noalloc.argtypes = [dp, P, P, P, P, i64p, i64p, i64p, P, P, P]
+    lib.fa_fwd_noalloc.restype = st
     _lib = lib
     return lib
 
 
 EXPORTED = ("fa_create", "fa_fwd", "fa_sync_status", "fa_destroy", "fa_last_error",
-            "fa_version", "fa_validate", "fa_visible_pairs", "fa_tile_class", "fa_plan_stats")
+            "fa_version", "fa_validate", "fa_visible_pairs", "fa_tile_class", "fa_plan_stats",
+            "fa_fwd_noalloc")
 
 
 def _check(status):
@@ -202,6 +205,22 @@ def fa_fwd(h, q, k, v, o, lse, atten_mask=None, prefix=None, actual_seq_qlen=Non
     a = _Arrays(prefix, actual_seq_qlen, actual_seq_kvlen)
     _check(load_library().fa_fwd(h, _ptr(q), _ptr(k), _ptr(v), _ptr(atten_mask), *a.ptrs(),
                                  _ptr(o), _ptr(lse), ctypes.c_void_p(int(stream))))
+
+
+def fa_fwd_noalloc(desc, q, k, v, o, lse, atten_mask=None, prefix=None, actual_seq_qlen=None,
+                   actual_seq_kvlen=None, stream=None):
+    """The allocation-free forward: no handle, the work list lives in the
+    library's fixed device array (see include/fa.h). Same arguments as
+    fa_fwd plus the descriptor."""
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    elif hasattr(stream, "cuda_stream"):
+        stream = stream.cuda_stream
+    a = _Arrays(prefix, actual_seq_qlen, actual_seq_kvlen)
+    _check(load_library().fa_fwd_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v),
+                                         _ptr(atten_mask), *a.ptrs(), _ptr(o), _ptr(lse),
+                                         ctypes.c_void_p(int(stream))))
 
 
 # ---------------------------------------------------------------- helper class

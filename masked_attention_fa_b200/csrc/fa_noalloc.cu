@@ -1,0 +1,277 @@
+// fa_fwd_noalloc: the forward for callers that must not allocate memory.
+//
+// Who needs this: code that runs where allocating is not allowed or not
+// safe, for example inside a framework that owns all device memory through
+// its own pool and forbids cudaMalloc/cudaFree behind its back, a real-time
+// inference loop that must not allocate after start-up, or a plugin that is
+// called from inside another library's allocator or memory callbacks. The
+// handle-based fa_create/fa_fwd path allocates a device workspace (and pinned
+// staging memory) for its work list; this entry point instead keeps the work
+// list and the error word in a fixed, file-scope device array that exists
+// from the moment the library is loaded onto a device until the process exits.
+//
+// Limits and sharing:
+//   - The array holds kNoAllocScratchBytes (1 MiB): a 256-byte header (error
+//     word), the per-sequence records (32 bytes per sequence, rounded up to
+//     256 bytes) and the work list (16 bytes per (sequence, head, block of
+//     256 query rows)). Larger problems are rejected with FA_ERR_UNSUPPORTED
+//     before any device work.
+//   - Every call, on every stream, shares the one array per device and leaves
+//     its own work list in it. Calls whose kernels overlap on the GPU (for
+//     example on two streams without ordering between them) race on the
+//     array; order them on one stream, or use fa_create/fa_fwd handles.
+//   - The first call on a device does the per-device set-up (it looks up the
+//     array's device address with cudaGetSymbolAddress, reads the device's
+//     attributes and sets the kernel's shared-memory attribute). Make that
+//     first call before any stream capture begins.
+//   - No cudaMalloc, cudaFree, pinned or host-heap allocation happens on the
+//     success path: the work list is built in a static host buffer, copied
+//     with cudaMemcpyAsync from pageable memory (the call returns once the
+//     driver has taken the bytes) and the error word is cleared with
+//     cudaMemsetAsync. Host calls are serialised by a mutex.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "fa_kernel.h"
+#include "fa_plan.h"
+
+// Size of the fixed device array (and of its host image).
+#define FA_NOALLOC_SCRATCH_BYTES (1u << 20)
+
+// The device scratch: header | SeqRec[B] | WorkItem[n]. In host code this
+// name denotes a host-side shadow, never a device address: the address that
+// kernels get comes from cudaGetSymbolAddress at set-up.
+static __device__ __align__(256) unsigned char g_fa_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+namespace fa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = FA_NOALLOC_SCRATCH_BYTES;
+constexpr size_t kNoAllocHeaderBytes = 256;
+constexpr int kNoAllocMaxDevices = 64;
+
+// Host copy of the same layout, filled before each upload.
+alignas(256) unsigned char g_host_image[kNoAllocScratchBytes];
+std::mutex g_mutex;
+
+struct DeviceSlot {
+  bool ready;
+  void* scratch;  // device address of g_fa_noalloc_scratch on that device
+  int num_sms;
+};
+DeviceSlot g_devices[kNoAllocMaxDevices];
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+fa_status_t cuda_err(cudaError_t e, const char* what) {
+  return fail(FA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Per-device set-up, once per device, with that device current.
+fa_status_t device_slot(DeviceSlot** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_err(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return fail(FA_ERR_UNSUPPORTED, "device index %d beyond %d", dev, kNoAllocMaxDevices);
+  DeviceSlot& s = g_devices[dev];
+  if (!s.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_err(e, "cudaDeviceGetAttribute");
+    if (major != 10 || minor != 0)
+      return fail(FA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library runs on sm_100 (B200)",
+                  dev, major, minor);
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_fa_noalloc_scratch);
+    if (e != cudaSuccess || ptr == nullptr)
+      return cuda_err(e == cudaSuccess ? cudaErrorInvalidSymbol : e, "cudaGetSymbolAddress");
+    s.scratch = ptr;
+    s.num_sms = sms;
+    s.ready = true;
+  }
+  *out = &s;
+  return FA_OK;
+}
+
+void strides_of(const fa_desc_t* d, int64_t S, int64_t* sb, int64_t* sh, int64_t* st) {
+  const int64_t N = d->N, D = d->D;
+  if (d->layout == FA_BNSD) {
+    *sb = N * S * D, *sh = S * D, *st = D;
+  } else if (d->layout == FA_BSND) {
+    *sb = S * N * D, *sh = D, *st = N * D;
+  } else {
+    *sb = 0, *sh = D, *st = N * D;
+  }
+}
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" fa_status_t fa_fwd_noalloc(const fa_desc_t* desc, const void* q, const void* k,
+                                      const void* v, const uint8_t* atten_mask,
+                                      const int64_t* prefix, const int64_t* actual_seq_qlen,
+                                      const int64_t* actual_seq_kvlen, void* o, float* lse,
+                                      void* cuda_stream) {
+  clear_error();
+  if (!desc) return fail(FA_ERR_NULLPTR, "desc is NULL");
+  if (!q || !k || !v || !o || !lse) return fail(FA_ERR_NULLPTR, "q, k, v, o and lse are required");
+  const int has_mask = (desc->sparse_mode <= 1) && atten_mask != nullptr;
+  fa_status_t st = validate_call(desc, prefix, actual_seq_qlen, actual_seq_kvlen, has_mask);
+  if (st != FA_OK) return st;
+  const uintptr_t align = (uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)o;
+  if (align & 15u) return fail(FA_ERR_PARAM_INVALID, "q, k, v and o must be 16-byte aligned");
+  if ((uintptr_t)lse & 3u) return fail(FA_ERR_PARAM_INVALID, "lse must be 4-byte aligned");
+
+  // Size of the work list, checked against the fixed array before anything else.
+  size_t n_items = 0;
+  for (int64_t b = 0; b < desc->B; ++b) {
+    int64_t sq = desc->Sq;
+    if (desc->layout == FA_TND) sq = actual_seq_qlen[b] - (b ? actual_seq_qlen[b - 1] : 0);
+    if (sq > 0) n_items += (size_t)((sq + kBlockM - 1) / kBlockM) * (size_t)desc->N;
+  }
+  const size_t seq_bytes = round256((size_t)desc->B * sizeof(SeqRec));
+  const size_t need = kNoAllocHeaderBytes + seq_bytes + n_items * sizeof(WorkItem);
+  if (need > kNoAllocScratchBytes)
+    return fail(FA_ERR_UNSUPPORTED,
+                "fa_fwd_noalloc: the work list needs %zu bytes but its fixed device array holds "
+                "%zu (%lld sequences, %zu work items); use fa_create/fa_fwd for this problem",
+                need, kNoAllocScratchBytes, (long long)desc->B, n_items);
+  if (n_items == 0) return FA_OK;
+
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceSlot* slot = nullptr;
+  st = device_slot(&slot);
+  if (st != FA_OK) return st;
+
+  // Per-sequence records and work items, built in the static host image with
+  // the same rules and order as the handle path.
+  SeqRec* recs = reinterpret_cast<SeqRec*>(g_host_image + kNoAllocHeaderBytes);
+  WorkItem* items = reinterpret_cast<WorkItem*>(g_host_image + kNoAllocHeaderBytes + seq_bytes);
+  int64_t first_ne = -1, last_ne = -1;
+  for (int64_t b = 0; b < desc->B; ++b) {
+    int64_t sq = desc->Sq;
+    if (desc->layout == FA_TND) sq = actual_seq_qlen[b] - (b ? actual_seq_qlen[b - 1] : 0);
+    if (sq > 0) {
+      if (first_ne < 0) first_ne = b;
+      last_ne = b;
+    }
+  }
+  for (int64_t b = 0; b < desc->B; ++b) {
+    int64_t qo = 0, ko = 0, sq = desc->Sq, skv = desc->Skv;
+    if (desc->layout == FA_TND) {
+      qo = b ? actual_seq_qlen[b - 1] : 0;
+      ko = b ? actual_seq_kvlen[b - 1] : 0;
+      sq = actual_seq_qlen[b] - qo;
+      skv = actual_seq_kvlen[b] - ko;
+    }
+    const __int128 delta = (__int128)skv - sq;
+    auto clampo = [](__int128 x) -> int64_t {
+      return x < -(__int128)kUnbounded ? -kUnbounded
+                                       : (x > (__int128)kUnbounded ? kUnbounded : (int64_t)x);
+    };
+    int64_t lo = -kUnbounded, hi = kUnbounded, pfx = 0;
+    int rule = desc->sparse_mode;
+    if (rule == 7) rule = (b == last_ne) ? 4 : 3;
+    if (rule == 8) rule = (b == first_ne) ? 4 : 2;
+    if (rule == 0 && has_mask) {  // band from the top-left
+      lo = clampo(-(__int128)desc->pre_tokens);
+      hi = clampo((__int128)desc->next_tokens);
+    } else if (rule == 2) {  // leftUpCausal
+      hi = 0;
+    } else if (rule == 3) {  // rightDownCausal
+      hi = clampo(delta);
+    } else if (rule == 4) {  // band from the bottom-right
+      lo = clampo(delta - desc->pre_tokens);
+      hi = clampo(delta + desc->next_tokens);
+    } else if (rule == 5 || rule == 6) {  // rightDownCausal plus prefix columns
+      hi = clampo(delta);
+      pfx = prefix[b];
+    }
+    recs[b] = SeqRec{(int32_t)qo, (int32_t)ko, (int32_t)sq, (int32_t)skv, (int32_t)lo, (int32_t)hi,
+                     (int32_t)pfx,
+                     (desc->sparse_mode == 1 || (desc->sparse_mode == 0 && has_mask))
+                         ? (int32_t)kSeqDenseMask : 0};
+  }
+  size_t n = 0;
+  for (int64_t b = 0; b < desc->B; ++b) {
+    const SeqRec& s = recs[b];
+    if (s.sq <= 0) continue;
+    const int32_t nblk = (s.sq + kBlockM - 1) / kBlockM;
+    for (int32_t qb = 0; qb < nblk; ++qb) {
+      int32_t cost = 0;
+      for (int sub = 0; sub < kSubTiles; ++sub) {
+        const TileRange t = tile_range(s, (int64_t)qb * kBlockM + sub * kTileM);
+        cost += t.hi > t.lo ? t.hi - t.lo : 0;
+      }
+      for (int64_t h = 0; h < desc->N; ++h) items[n++] = WorkItem{(int32_t)b, (int32_t)h, qb, cost};
+    }
+  }
+  // Descending cost, ties in generation order (b, block, head): the same
+  // order a stable sort by cost gives, without a temporary buffer.
+  std::sort(items, items + n, [](const WorkItem& a, const WorkItem& c) {
+    if (a.cost != c.cost) return a.cost > c.cost;
+    if (a.b != c.b) return a.b < c.b;
+    if (a.qblk != c.qblk) return a.qblk < c.qblk;
+    return a.h < c.h;
+  });
+
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  unsigned char* dscr = static_cast<unsigned char*>(slot->scratch);
+  cudaError_t e = cudaMemsetAsync(dscr, 0, kNoAllocHeaderBytes, stream);  // error word = 0
+  if (e != cudaSuccess) return cuda_err(e, "cudaMemsetAsync");
+  e = cudaMemcpyAsync(dscr + kNoAllocHeaderBytes, g_host_image + kNoAllocHeaderBytes,
+                      need - kNoAllocHeaderBytes, cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return cuda_err(e, "cudaMemcpyAsync");
+
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  const fa_desc_t* d = desc;
+  const bool tnd = d->layout == FA_TND;
+  const void* ptrs[3] = {q, k, v};
+  CUtensorMap* maps[3] = {&p.tm_q, &p.tm_k, &p.tm_v};
+  for (int i = 0; i < 3; ++i) {
+    const int64_t S = i == 0 ? d->Sq : d->Skv;
+    int64_t sb, sh, stt;
+    strides_of(d, S, &sb, &sh, &stt);
+    const int64_t b_stride = tnd ? (S > 0 ? S : 1) * d->N * d->D : sb;
+    if (!encode_operand_map(maps[i], ptrs[i], d->D, S, d->N, tnd ? 1 : d->B, stt, sh, b_stride))
+      return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed for operand %d", i);
+  }
+  p.err_word = reinterpret_cast<unsigned int*>(dscr);
+  p.seqs = reinterpret_cast<const SeqRec*>(dscr + kNoAllocHeaderBytes);
+  p.items = reinterpret_cast<const WorkItem*>(dscr + kNoAllocHeaderBytes + seq_bytes);
+  p.o = o;
+  p.lse = lse;
+  p.mask = atten_mask;
+  strides_of(d, d->Sq, &p.o_sb, &p.o_sh, &p.o_st);
+  p.l_sb = tnd ? 0 : d->N * d->Sq;
+  p.l_sh = d->Sq;
+  if (has_mask) {
+    const int64_t plane = d->Sq * d->Skv;
+    p.m_si = d->Skv;
+    p.m_sb = (d->mask_kind == FA_MASK_SS) ? 0 : (d->mask_kind == FA_MASK_B1SS ? plane : d->N * plane);
+    p.m_sh = (d->mask_kind == FA_MASK_BNSS) ? plane : 0;
+  }
+  p.n_items = (int32_t)n;
+  p.tnd = tnd ? 1 : 0;
+  p.scale_log2 = (float)(d->scale * 1.4426950408889634073599);
+  p.debug_flags = 0;
+  p.timeout_ns = 2000000000ull;
+  const int grid = (int)std::min<size_t>(n, (size_t)slot->num_sms);
+  const char* why = nullptr;
+  e = launch_fwd((int)d->D, p, grid, stream, &why);
+  if (e != cudaSuccess) {
+    if (why) return fail(FA_ERR_UNSUPPORTED, "launch refused: %s", why);
+    return cuda_err(e, "kernel launch");
+  }
+  return FA_OK;
+}
