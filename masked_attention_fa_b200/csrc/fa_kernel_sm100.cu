@@ -10,15 +10,15 @@
 // One persistent CTA per SM, 16 warps, warp-specialised:
 //   warps 0-3   softmax of query sub-tile 0 (rows 0..127 of the item)
 //   warps 4-7   softmax of query sub-tile 1 (rows 128..255)
-//   warp 12     tcgen05.mma issuer (one thread)
+//   warp 12     tcgen05.mma issuer (one thread; owns TMEM)
 //   warp 13     TMA producer (one thread)
 //   other warps idle (they give their registers to the softmax warps)
 // Tensor memory (512 columns): S0 | S1 | O0 | O1. S_s holds the fp32 scores
 // of sub-tile s; the softmax overwrites its first 64 columns with P (bf16
 // pairs), which feeds the P.V MMA directly from TMEM. O_s accumulates fp32.
 // MMA issue order per key tile t:  PV0(t), QK0(t+1), PV1(t), QK1(t+1), so
-// each softmax warpgroup has the time of two MMAs to turn S into P, and
-// every S_s(t+1) commit also proves PV_s(t) complete (commits track all
+// each softmax warpgroup has the time of two MMA groups to turn S into P,
+// and every S_s(t+1) commit also proves PV_s(t) complete (commits track all
 // earlier MMAs), which is what lets the softmax rescale O_s in place.
 // Every mbarrier wait is bounded (globaltimer); on expiry the CTA records
 // the site in the error word, drains its in-flight copies and MMAs, frees
@@ -39,11 +39,16 @@ namespace dev {
 constexpr int kThreads = 512;
 constexpr int kWarpMma = 12;
 constexpr int kWarpLoad = 13;
-constexpr int kRegsSoftmax = 208;  // 2 warpgroups x 128 threads x 208
-constexpr int kRegsOther = 48;     // + 2 warpgroups x 128 threads x 48 = 512 x 128
-static_assert(2 * 128 * kRegsSoftmax + 2 * 128 * kRegsOther == kThreads * 128,
-              "register split must equal the launch allocation");
+// Register split (setmaxnreg) over the 512 x 128 registers of the launch:
+// softmax warpgroups 0-1 take 208, the idle warpgroup 2 keeps 24, the
+// warpgroup of the MMA and TMA warps keeps 72.
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsIdle = 24;
+constexpr int kRegsControl = 72;
+constexpr int kRegsTotal = 2 * 128 * kRegsSoftmax + 128 * kRegsIdle + 128 * kRegsControl;
+static_assert(kRegsTotal == kThreads * 128, "register split must equal the launch allocation");
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
+constexpr int kPChunks = 4;           // P is exponentiated and stored 32 keys at a time
 
 // Where a wait gave up (error word bits 8..15).
 enum WaitSite : uint32_t {
@@ -73,7 +78,7 @@ struct Ctl {
   uint64_t q_full, q_empty;
   uint64_t kv_full[NS], kv_empty[NS];
   uint64_t s_full[2], p_full[2], o_done[2];
-  uint64_t drain;
+  uint64_t drain[1];
   uint32_t tmem_base;
   volatile int abort_flag;
 };
@@ -101,6 +106,108 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// Three-input maximum (sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t pack_f32x2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// (a, b) <- (a, b) * m2 + c2, two lanes per instruction.
+__device__ __forceinline__ void fma_x2(float& a, float& b, uint64_t m2, uint64_t c2) {
+  asm("{\n\t.reg .b64 r;\n\t"
+      "mov.b64 r, {%0, %1};\n\t"
+      "fma.rn.f32x2 r, r, %2, %3;\n\t"
+      "mov.b64 {%0, %1}, r;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "l"(m2), "l"(c2));
+}
+
+// (a, b) += (x, y), two lanes per instruction.
+__device__ __forceinline__ void add_x2(float& a, float& b, float x, float y) {
+  asm("{\n\t.reg .b64 r, s;\n\t"
+      "mov.b64 r, {%0, %1};\n\t"
+      "mov.b64 s, {%2, %3};\n\t"
+      "add.rn.f32x2 r, r, s;\n\t"
+      "mov.b64 {%0, %1}, r;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "f"(x), "f"(y));
+}
+
+// 2^x for two values on the FMA pipe instead of the MUFU unit. Cody-Waite
+// reduction x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the
+// low mantissa bits), a degree-3 minimax polynomial for 2^f on [-1/2, 1/2]
+// (Remez, relative error 7.5e-5; coefficients from gen_exp2_poly.py), and n
+// added into the exponent field. Inputs are clamped to >= -126.
+__device__ __forceinline__ void ex2_poly_x2(float& a, float& b) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  a = fmaxf(a, -126.0f);
+  b = fmaxf(b, -126.0f);
+  float ta = a, tb = b;
+  add_x2(ta, tb, kShift, kShift);   // t = x + shift (rounded: n in the low bits)
+  float na = ta, nb = tb;
+  add_x2(na, nb, -kShift, -kShift); // n = t - shift
+  float fa = -na, fb = -nb;
+  add_x2(fa, fb, a, b);             // f = x - n, |f| <= 1/2
+  float pa = 0.05517167f, pb = 0.05517167f;
+  fma_x2(pa, pb, pack_f32x2(fa, fb), pack_f32x2(0.24261113f, 0.24261113f));
+  fma_x2(pa, pb, pack_f32x2(fa, fb), pack_f32x2(0.69326097f, 0.69326097f));
+  fma_x2(pa, pb, pack_f32x2(fa, fb), pack_f32x2(0.99992806f, 0.99992806f));
+  a = __int_as_float(__float_as_int(pa) + (__float_as_int(ta) << 23));
+  b = __int_as_float(__float_as_int(pb) + (__float_as_int(tb) << 23));
+}
+
+// Columns c with (c % 8) < kPolyPer8 take the FMA-pipe exponential on tiles
+// without masked entries; the rest use ex2.approx on the MUFU unit.
+constexpr int kPolyPer8 = 0;
+
+// Row maximum of 128 scores: eight independent chains of 3-input maxima.
+__device__ __forceinline__ float row_max128(const float (&x)[128]) {
+  float m[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    float a = x[j];
+#pragma unroll
+    for (int r = 1; r < 15; r += 2) a = max3f(a, x[8 * r + j], x[8 * (r + 1) + j]);
+    m[j] = fmaxf(a, x[120 + j]);
+  }
+  return max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+}
+
+// x <- 2^(x * scale_log2 - ref) in place; returns the row sum (eight
+// independent partial sums). kPoly: some columns use ex2_poly_x2.
+template <bool kPoly>
+__device__ __forceinline__ float exp_rows(float (&x)[128], float scale_log2, float ref) {
+  const uint64_t m2 = pack_f32x2(scale_log2, scale_log2);
+  const uint64_t c2 = pack_f32x2(-ref, -ref);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c = 0; c < 128; c += 2) {
+    float a = x[c], b = x[c + 1];
+    fma_x2(a, b, m2, c2);
+    if (kPoly && (c & 7) < kPolyPer8) {
+      ex2_poly_x2(a, b);
+    } else {
+      a = ex2(a);
+      b = ex2(b);
+    }
+    x[c] = a;
+    x[c + 1] = b;
+    const int k = (c >> 1) & 3;
+    add_x2(acc[2 * k], acc[2 * k + 1], a, b);
+  }
+  add_x2(acc[0], acc[1], acc[2], acc[3]);
+  add_x2(acc[4], acc[5], acc[6], acc[7]);
+  add_x2(acc[0], acc[1], acc[4], acc[5]);
+  return acc[0] + acc[1];
 }
 
 // ----------------------------------------------------------------- mbarrier
@@ -350,20 +457,27 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem, const uint8_t* sQ, const
 }
 
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t tmem, const uint8_t* sKV, int sub,
-                                         uint32_t vst, bool accumulate) {
+__device__ __forceinline__ void issue_pv(uint32_t tmem, const uint8_t* sKV, int sub, uint32_t vst,
+                                         bool accumulate) {
   using C = Cfg<D>;
   constexpr uint32_t idesc = idesc_bf16(128, D, true);
   // V is MN-major (D contiguous): step k moves 16 key rows = 2048 bytes.
   const uint64_t b0 = sdesc(smem_u32(sKV) + vst * C::kTileBytes, C::kChunkBytes, 1024u);
   const uint32_t a = tmem + C::col_s(sub);  // P: 128 bf16 = 64 columns
   const uint32_t d = tmem + C::col_o(sub);
-#pragma unroll 1
+#pragma unroll
   for (int k = 0; k < kTileN / 16; ++k)
     mma_ts(d, a + k * 8u, b0 + (uint64_t)(k * (2048u >> 4)), idesc,
            (accumulate || k > 0) ? 1u : 0u);
 }
 
+// MMA issue (one thread). Per key tile t, in this order:
+//   O_0 += P_0(t) V(t); S_0(t+1) = Q_0 K(t+1)^T; O_1 += P_1(t) V(t);
+//   S_1(t+1) = Q_1 K(t+1)^T
+// so each softmax warpgroup has two MMA groups' time to turn S into P. Both
+// ring waits come before the first group and the commits follow the QK
+// groups, so consecutive groups go out with only the P wait between them:
+// the tensor pipe queues few instructions and any gap in issue idles it.
 template <int D>
 __device__ void mma_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t tmem,
                          const uint8_t* sQ, const uint8_t* sKV, const WaitCtx& w) {
@@ -384,15 +498,12 @@ __device__ void mma_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t
       break;
     }
     ++q_loads;
-    tc_fence_after();
-    // First K tile: both sub-tiles' QK.
     uint32_t kst = ring % NS;
     if (!wait_bounded(&ctl->kv_full[kst], (ring / NS) & 1u, w, kSiteKvFull)) {
       ok = false;
       break;
     }
     ++ring;
-    tc_fence_after();
 #pragma unroll
     for (int s = 0; s < 2; ++s)
       if (active(ip.tr[s], ip.lo)) {
@@ -402,26 +513,14 @@ __device__ void mma_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t
     mma_commit(&ctl->kv_empty[kst]);
     if (ip.lo + 1 == ip.hi) mma_commit(&ctl->q_empty);
     bool first[2] = {true, true};
-    for (int t = ip.lo; t < ip.hi; ++t) {
+    for (int t = ip.lo; t < ip.hi && ok; ++t) {
       const uint32_t vst = ring % NS;
       if (!wait_bounded(&ctl->kv_full[vst], (ring / NS) & 1u, w, kSiteKvFull)) {
         ok = false;
         break;
       }
       ++ring;
-      tc_fence_after();
       const bool nxt = t + 1 < ip.hi;
-      if (active(ip.tr[0], t)) {
-        if (!wait_bounded(&ctl->p_full[0], p_count[0] & 1u, w, kSitePFull)) {
-          ok = false;
-          break;
-        }
-        ++p_count[0];
-        tc_fence_after();
-        issue_pv<D>(tmem, sKV, 0, vst, !first[0]);
-        first[0] = false;
-        if (t == ip.tr[0].hi - 1) mma_commit(&ctl->o_done[0]);
-      }
       if (nxt) {
         kst = ring % NS;
         if (!wait_bounded(&ctl->kv_full[kst], (ring / NS) & 1u, w, kSiteKvFull)) {
@@ -429,29 +528,28 @@ __device__ void mma_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t
           break;
         }
         ++ring;
-        tc_fence_after();
-        if (active(ip.tr[0], t + 1)) {
-          issue_qk<D>(tmem, sQ, sKV, 0, kst);
-          mma_commit(&ctl->s_full[0]);
+      }
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        if (active(ip.tr[s], t)) {
+          if (!wait_bounded(&ctl->p_full[s], p_count[s] & 1u, w, kSitePFull)) {
+            ok = false;
+            break;
+          }
+          ++p_count[s];
+          tc_fence_after();
+          issue_pv<D>(tmem, sKV, s, vst, !first[s]);
+          first[s] = false;
+          if (t == ip.tr[s].hi - 1) mma_commit(&ctl->o_done[s]);
+        }
+        if (nxt && active(ip.tr[s], t + 1)) {
+          issue_qk<D>(tmem, sQ, sKV, s, kst);
+          mma_commit(&ctl->s_full[s]);
         }
       }
-      if (active(ip.tr[1], t)) {
-        if (!wait_bounded(&ctl->p_full[1], p_count[1] & 1u, w, kSitePFull)) {
-          ok = false;
-          break;
-        }
-        ++p_count[1];
-        tc_fence_after();
-        issue_pv<D>(tmem, sKV, 1, vst, !first[1]);
-        first[1] = false;
-        if (t == ip.tr[1].hi - 1) mma_commit(&ctl->o_done[1]);
-      }
+      if (!ok) break;
       mma_commit(&ctl->kv_empty[vst]);
       if (nxt) {
-        if (active(ip.tr[1], t + 1)) {
-          issue_qk<D>(tmem, sQ, sKV, 1, kst);
-          mma_commit(&ctl->s_full[1]);
-        }
         mma_commit(&ctl->kv_empty[kst]);
         if (t + 2 == ip.hi) mma_commit(&ctl->q_empty);
       }
@@ -459,9 +557,69 @@ __device__ void mma_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t
   }
   if (!ok) {
     // Abort: wait until every MMA issued so far has finished with TMEM/SMEM.
-    mma_commit(&ctl->drain);
-    wait_bounded(&ctl->drain, 0u, w, kSiteDrain, false);
+    mma_commit(&ctl->drain[0]);
+    wait_bounded(&ctl->drain[0], 0u, w, kSiteDrain, false);
   }
+}
+
+// Scores of this thread's row (128 keys of S_s) with the element mask of a
+// boundary tile applied (-inf where the key is not visible).
+__device__ __forceinline__ void load_scores(uint32_t tS, float (&x)[128], bool partial, int c_lo,
+                                            int c_hi, const uint32_t (&mbits)[4]) {
+  uint32_t sv[128];
+  tmem_ld128_wait(tS, sv);
+#pragma unroll
+  for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sv[c]);
+  if (partial) {
+#pragma unroll
+    for (int c = 0; c < 128; ++c)
+      if (c < c_lo || c > c_hi || ((mbits[c >> 5] >> (c & 31)) & 1u)) x[c] = -INFINITY;
+  }
+}
+
+// Exponentiate keys [32 c, 32 c + 32) of the row against `ref`, add them to
+// the eight partial sums and pack P into 16 bf16 pairs.
+template <bool kPoly>
+__device__ __forceinline__ void exp_chunk(float (&x)[128], int chunk, uint64_t m2, uint64_t c2,
+                                          float (&acc)[8], uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    const int c = chunk * 32 + j;
+    float a = x[c], b = x[c + 1];
+    fma_x2(a, b, m2, c2);
+    if (kPoly && (c & 7) < kPolyPer8) {
+      ex2_poly_x2(a, b);
+    } else {
+      a = ex2(a);
+      b = ex2(b);
+    }
+    const int k = (j >> 1) & 3;
+    add_x2(acc[2 * k], acc[2 * k + 1], a, b);
+    pk[j >> 1] = pack_bf16(a, b);
+  }
+}
+
+// Exponentiate the row chunk by chunk, storing each chunk of P as soon as it
+// is packed; one arrival on p_full once every store has landed.
+template <bool kPoly>
+__device__ __forceinline__ float exp_store_p(float (&x)[128], float scale_log2, float ref,
+                                             uint32_t tS, uint64_t* p_full) {
+  const uint64_t m2 = pack_f32x2(scale_log2, scale_log2);
+  const uint64_t c2 = pack_f32x2(-ref, -ref);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c = 0; c < kPChunks; ++c) {
+    uint32_t pk[16];
+    exp_chunk<kPoly>(x, c, m2, c2, acc, pk);
+    tmem_st16(tS + 16u * c, pk);
+  }
+  tmem_st_wait();
+  tc_fence_before();
+  mbar_arrive(p_full);
+  add_x2(acc[0], acc[1], acc[2], acc[3]);
+  add_x2(acc[4], acc[5], acc[6], acc[7]);
+  add_x2(acc[0], acc[1], acc[4], acc[5]);
+  return acc[0] + acc[1];
 }
 
 template <int D>
@@ -519,20 +677,9 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint
         }
       }
       tc_fence_after();
-      uint32_t sv[128];
-      tmem_ld128_wait(tS, sv);
       float x[128];
-#pragma unroll
-      for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sv[c]);
-      if (partial) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c < c_lo || c > c_hi || ((mbits[c >> 5] >> (c & 31)) & 1u)) x[c] = -INFINITY;
-      }
-      float mb = x[0];
-#pragma unroll
-      for (int c = 1; c < 128; ++c) mb = fmaxf(mb, x[c]);
-      const float m_new = mb * scale_log2;
+      load_scores(tS, x, partial, c_lo, c_hi, mbits);
+      const float m_new = row_max128(x) * scale_log2;
       const bool resc = m_new > m_used + kRescaleLog2;
       float alpha = 1.f;
       if (resc) {
@@ -540,24 +687,10 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint
         l *= alpha;
         m_used = m_new;
       }
-      const float ref = (m_used == -INFINITY) ? 0.f : m_used;
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        x[c] = ex2(fmaf(x[c], scale_log2, -ref));
-        sum += x[c];
-      }
-      l += sum;
-      uint32_t pk[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(x[2 * c], x[2 * c + 1]);
-      tmem_st32(tS, pk);
-#pragma unroll
-      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(x[64 + 2 * c], x[64 + 2 * c + 1]);
-      tmem_st32(tS + 32u, pk);
       // O_s already holds PV(t-1) (the S_s(t) commit tracked it); rescale it
-      // in place when this row's reference max moved. Not on the item's
-      // first tile: its PV overwrites O_s.
+      // in place when this row's reference max moved, before the first P
+      // chunk lets PV(t) accumulate. Not on the item's first tile: its PV
+      // overwrites O_s.
       if (t > tr.lo && __any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
         for (int ch = 0; ch < D / 32; ++ch) {
@@ -568,9 +701,9 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint
           tmem_st32(tO + ch * 32u, ov);
         }
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&ctl->p_full[sub]);
+      const float ref = (m_used == -INFINITY) ? 0.f : m_used;
+      l += partial ? exp_store_p<false>(x, scale_log2, ref, tS, &ctl->p_full[sub])
+                   : exp_store_p<true>(x, scale_log2, ref, tS, &ctl->p_full[sub]);
     }
     if (!ok) break;
     // Epilogue: O / l -> bf16, lse = ln(sum exp(scale q.k)).
@@ -635,7 +768,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100(const __grid_constan
       mbar_init(&ctl->p_full[s], 128);
       mbar_init(&ctl->o_done[s], 1);
     }
-    mbar_init(&ctl->drain, 1);
+    mbar_init(&ctl->drain[0], 1);
     ctl->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -656,8 +789,10 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100(const __grid_constan
   if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     softmax_role<D>(p, ctl, tmem, warp >> 2, w);
+  } else if (warp < 12) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsIdle));
   } else {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
     if (warp == kWarpMma && lane == 0) mma_role<D>(p, ctl, tmem, sQ, sKV, w);
     if (warp == kWarpLoad && lane == 0) load_role<D>(p, ctl, sQ, sKV, w);
   }
@@ -724,7 +859,7 @@ static cudaError_t launch_d(const FwdParams& p, int grid, cudaStream_t stream, c
     if (e != cudaSuccess) return e;
     // setmaxnreg redistributes the registers the CTA was launched with; a
     // split larger than that allocation would never be granted.
-    regs_ok = attr.numRegs * dev::kThreads >= 2 * 128 * dev::kRegsSoftmax + 2 * 128 * dev::kRegsOther;
+    regs_ok = attr.numRegs * dev::kThreads >= dev::kRegsTotal;
     configured = true;
   }
   if (!regs_ok) {
