@@ -62,13 +62,21 @@ def load_peaks():
 
 
 def load_traffic(workload):
-    """Per-launch DRAM bytes of the main kernel from the committed ncu summary."""
+    """Per-launch DRAM bytes (read + write) of the main kernel from the committed
+    ncu summary; None when the kernel source changed since that capture."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "masked_attention_fa_b200", "csrc", "fa_kernel_sm100.cu")
     try:
         with open(path) as f:
-            return json.load(f).get(workload)
+            rec = json.load(f)
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
     except (OSError, ValueError):
         return None
+    if rec.get("kernel_source_sha256") != sha or workload not in rec:
+        return None
+    return rec[workload].get("dram_bytes_per_launch")
 
 
 class ClockSampler:
