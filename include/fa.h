@@ -227,6 +227,41 @@ fa_status_t fa_plan_stats(const fa_desc_t* desc, const int64_t* prefix,
                           const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
                           int32_t has_mask, int64_t* out);
 
+/* ---------------- query split across devices (host only) ---------------- */
+
+/* One part of a query split: its own problem and where it sits in the
+ * unsplit tensors. */
+typedef struct {
+    fa_desc_t desc;            /* the part's problem: TND, sparse_mode 7/3 or 8/2 */
+    int64_t q_begin, q_end;    /* its query tokens [q_begin, q_end) of the unsplit Q, O, lse */
+    int64_t kv_begin, kv_end;  /* its key tokens [kv_begin, kv_end) of the unsplit K, V */
+} fa_split_part_t;
+
+/*
+ * fa_split_queries — the multi-card scheme of the sparseMode page
+ * (sparseMode=7 / sparseMode=8 sections): the query tokens of a varlen job
+ * are cut into n_parts contiguous ranges, key/value are not cut, and each
+ * part becomes an independent call whose outputs are exactly the unsplit
+ * call's rows [q_begin, q_end). A rightDownCausal job (mode 3) gives parts in
+ * mode 7 (the last sequence of a part, cut at its top, is the band with
+ * preTokens = Skv_b, nextTokens = rows kept - Sq_b) or mode 3; a leftUpCausal
+ * job (mode 2) gives parts in mode 8 (the first sequence, cut at its bottom,
+ * is the band with preTokens = Skv_b, nextTokens = Sq_b - Skv_b for a bottom
+ * piece) or mode 2.
+ *
+ * desc: TND, sparse_mode 2 or 3 (mode 3 needs Sq_b <= Skv_b for every
+ * sequence, as the sparseMode=7 section requires of its non-band batches).
+ * cuts: host int64[n_parts - 1], increasing query-token positions in
+ * [0, T_q]; NULL = balance the visible-pair count of the parts.
+ * part: 0 .. n_parts-1. out: the part; out_seq_qlen / out_seq_kvlen: host
+ * int64[desc->B], receive the part's cumulative arrays (out->desc.B entries).
+ * An empty part has Sq = Skv = 0 and one empty sequence.
+ */
+fa_status_t fa_split_queries(const fa_desc_t* desc, const int64_t* actual_seq_qlen,
+                             const int64_t* actual_seq_kvlen, int32_t n_parts,
+                             const int64_t* cuts, int32_t part, fa_split_part_t* out,
+                             int64_t* out_seq_qlen, int64_t* out_seq_kvlen);
+
 #ifdef __cplusplus
 }
 #endif

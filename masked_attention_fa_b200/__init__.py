@@ -52,6 +52,16 @@ class fa_desc_t(ctypes.Structure):
     ]
 
 
+class fa_split_part_t(ctypes.Structure):
+    _fields_ = [
+        ("desc", fa_desc_t),
+        ("q_begin", ctypes.c_int64),
+        ("q_end", ctypes.c_int64),
+        ("kv_begin", ctypes.c_int64),
+        ("kv_end", ctypes.c_int64),
+    ]
+
+
 _lib = None
 
 
@@ -91,13 +101,16 @@ def load_library():
     lib.fa_plan_stats.restype = st
     lib.fa_fwd_noalloc.argtypes = [dp, P, P, P, P, i64p, i64p, i64p, P, P, P]
     lib.fa_fwd_noalloc.restype = st
+    lib.fa_split_queries.argtypes = [dp, i64p, i64p, ctypes.c_int32, i64p, ctypes.c_int32,
+                                     ctypes.POINTER(fa_split_part_t), i64p, i64p]
+    lib.fa_split_queries.restype = st
     _lib = lib
     return lib
 
 
 EXPORTED = ("fa_create", "fa_fwd", "fa_sync_status", "fa_destroy", "fa_last_error",
             "fa_version", "fa_validate", "fa_visible_pairs", "fa_tile_class", "fa_plan_stats",
-            "fa_fwd_noalloc")
+            "fa_fwd_noalloc", "fa_split_queries")
 
 
 def _check(status):
@@ -221,6 +234,28 @@ def fa_fwd_noalloc(desc, q, k, v, o, lse, atten_mask=None, prefix=None, actual_s
     _check(load_library().fa_fwd_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v),
                                          _ptr(atten_mask), *a.ptrs(), _ptr(o), _ptr(lse),
                                          ctypes.c_void_p(int(stream))))
+
+
+def fa_split_queries(desc, actual_seq_qlen, actual_seq_kvlen, n_parts, part, cuts=None):
+    """Part `part` of the query split of a TND mode-2/3 job (see include/fa.h).
+
+    Returns a dict with the part's descriptor, its query token range
+    [q_begin, q_end) and key range [kv_begin, kv_end) in the unsplit tensors,
+    and its cumulative length arrays.
+    """
+    a = _Arrays(None, actual_seq_qlen, actual_seq_kvlen)
+    c = None if cuts is None else np.ascontiguousarray(cuts, dtype=np.int64)
+    out = fa_split_part_t()
+    oq = np.zeros(int(desc.B), dtype=np.int64)
+    ok = np.zeros(int(desc.B), dtype=np.int64)
+    _, pq, pk = a.ptrs()
+    _check(load_library().fa_split_queries(
+        ctypes.byref(desc), pq, pk, int(n_parts), _Arrays._p(c), int(part), ctypes.byref(out),
+        _Arrays._p(oq), _Arrays._p(ok)))
+    nb = int(out.desc.B)
+    return {"desc": out.desc, "q_begin": int(out.q_begin), "q_end": int(out.q_end),
+            "kv_begin": int(out.kv_begin), "kv_end": int(out.kv_end),
+            "actual_seq_qlen": oq[:nb].tolist(), "actual_seq_kvlen": ok[:nb].tolist()}
 
 
 # ---------------------------------------------------------------- helper class

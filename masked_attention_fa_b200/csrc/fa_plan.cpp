@@ -12,6 +12,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstring>
 #include <string>
 
 namespace fa {
@@ -295,6 +296,135 @@ int32_t tile_class(const SeqRec& s, int64_t qt, int64_t kt) {
   return FA_TILE_PARTIAL;
 }
 
+
+// Query split across devices: see fa_split_queries in fa.h. The unsplit job
+// is TND in mode 2 or 3; a part keeps every key of the sequences it touches.
+static int64_t row_cost(int mode, int64_t i, int64_t sq, int64_t skv) {
+  // visible keys of row i: mode 3 sees j <= i + (skv - sq), mode 2 sees j <= i
+  const int64_t hi = (mode == 3) ? i + (skv - sq) : i;
+  return imax64(0, imin64(hi + 1, skv));
+}
+
+fa_status_t split_queries(const fa_desc_t* d, const int64_t* cu_q, const int64_t* cu_kv,
+                          int32_t n_parts, const int64_t* cuts, int32_t part,
+                          fa_split_part_t* out, int64_t* oq, int64_t* okv) {
+  if (!out || !oq || !okv) return fail(FA_ERR_NULLPTR, "out arrays are required");
+  fa_status_t st = validate_call(d, nullptr, cu_q, cu_kv, 0);
+  if (st != FA_OK) return st;
+  if (d->layout != FA_TND || (d->sparse_mode != 2 && d->sparse_mode != 3))
+    return fail(FA_ERR_UNSUPPORTED, "query split needs a TND job in sparse_mode 2 or 3");
+  if (n_parts < 1 || part < 0 || part >= n_parts)
+    return fail(FA_ERR_PARAM_INVALID, "part %d of %d parts", part, n_parts);
+  const int mode = d->sparse_mode;
+  const int64_t T = d->Sq;
+  auto seq = [&](int64_t b, int64_t* qo, int64_t* ko, int64_t* sq, int64_t* skv) {
+    *qo = b ? cu_q[b - 1] : 0;
+    *ko = b ? cu_kv[b - 1] : 0;
+    *sq = cu_q[b] - *qo;
+    *skv = cu_kv[b] - *ko;
+  };
+  if (mode == 3) {
+    for (int64_t b = 0; b < d->B; ++b) {
+      int64_t qo, ko, sq, skv;
+      seq(b, &qo, &ko, &sq, &skv);
+      if (sq > skv)
+        return fail(FA_ERR_UNSUPPORTED,
+                    "splitting a rightDownCausal job needs Sq_b <= Skv_b (sequence %lld)",
+                    (long long)b);
+    }
+  }
+  // The part's query tokens [a, e).
+  int64_t a = 0, e = T;
+  if (cuts) {
+    int64_t prev = 0;
+    for (int32_t k = 0; k + 1 < n_parts; ++k) {
+      if (cuts[k] < prev || cuts[k] > T)
+        return fail(FA_ERR_PARAM_INVALID, "cuts must be increasing positions in [0, T_q]");
+      prev = cuts[k];
+    }
+    a = part ? cuts[part - 1] : 0;
+    e = part + 1 < n_parts ? cuts[part] : T;
+  } else {
+    // Balance the visible pairs: cut where the running cost crosses k/n of it.
+    int64_t total = 0;
+    for (int64_t b = 0; b < d->B; ++b) {
+      int64_t qo, ko, sq, skv;
+      seq(b, &qo, &ko, &sq, &skv);
+      for (int64_t i = 0; i < sq; ++i) total += row_cost(mode, i, sq, skv);
+    }
+    auto cut_at = [&](int32_t k) -> int64_t {  // first token whose prefix cost >= k/n of total
+      if (k <= 0) return 0;
+      if (k >= n_parts) return T;
+      const __int128 target = (__int128)total * k;
+      __int128 run = 0;
+      for (int64_t b = 0; b < d->B; ++b) {
+        int64_t qo, ko, sq, skv;
+        seq(b, &qo, &ko, &sq, &skv);
+        for (int64_t i = 0; i < sq; ++i) {
+          if (run * n_parts >= target) return qo + i;
+          run += row_cost(mode, i, sq, skv);
+        }
+      }
+      return T;
+    };
+    a = cut_at(part);
+    e = cut_at(part + 1);
+  }
+  std::memset(out, 0, sizeof(*out));
+  out->desc = *d;
+  out->desc.sparse_mode = mode;
+  out->desc.pre_tokens = 0;
+  out->desc.next_tokens = 0;
+  out->q_begin = a;
+  out->q_end = e;
+  if (a >= e) {  // empty part
+    out->desc.B = 1;
+    out->desc.Sq = out->desc.Skv = 0;
+    out->kv_begin = out->kv_end = 0;
+    oq[0] = okv[0] = 0;
+    return FA_OK;
+  }
+  int64_t b0 = 0;
+  while (cu_q[b0] <= a) ++b0;  // sequence holding token a
+  int64_t b1 = b0;
+  while (cu_q[b1] < e) ++b1;   // sequence holding token e - 1
+  int64_t qo0, ko0, sq0, skv0, qo1, ko1, sq1, skv1;
+  seq(b0, &qo0, &ko0, &sq0, &skv0);
+  seq(b1, &qo1, &ko1, &sq1, &skv1);
+  int64_t nq = 0, nk = 0;
+  for (int64_t b = b0; b <= b1; ++b) {
+    int64_t qo, ko, sq, skv;
+    seq(b, &qo, &ko, &sq, &skv);
+    const int64_t r0 = imax64(a, qo) - qo, r1 = imin64(e, qo + sq) - qo;
+    nq += imax64(0, r1 - r0);
+    nk += skv;
+    oq[b - b0] = nq;
+    okv[b - b0] = nk;
+  }
+  out->desc.B = b1 - b0 + 1;
+  out->desc.Sq = nq;
+  out->desc.Skv = nk;
+  out->kv_begin = ko0;
+  out->kv_end = ko1 + skv1;
+  const int64_t c0 = a - qo0;             // first kept row of sequence b0
+  const int64_t c1 = imin64(e, qo1 + sq1) - qo1;  // one past the last kept row of b1
+  if (mode == 3 && c1 < sq1) {
+    // The last sequence keeps rows [.., c1) of a rightDownCausal block: a band
+    // anchored at the bottom-right with next = c1 - Sq_b, pre = Skv_b.
+    out->desc.sparse_mode = 7;
+    out->desc.pre_tokens = skv1;
+    out->desc.next_tokens = c1 - sq1;
+  } else if (mode == 2 && c0 > 0) {
+    // The first sequence keeps rows [c0, ..) of a leftUpCausal block: a band
+    // with next = (last kept row + 1) - Skv_b, pre = Skv_b.
+    const int64_t c0_end = (b0 == b1) ? c1 : sq0;
+    out->desc.sparse_mode = 8;
+    out->desc.pre_tokens = skv0;
+    out->desc.next_tokens = c0_end - skv0;
+  }
+  return validate_call(&out->desc, nullptr, oq, okv, 0);
+}
+
 }  // namespace fa
 
 using namespace fa;
@@ -337,6 +467,15 @@ int32_t fa_tile_class(const fa_desc_t* desc, const int64_t* prefix,
   }
   auto recs = decode_geometry(desc, prefix, actual_seq_qlen, actual_seq_kvlen, has_mask);
   return tile_class(recs[(size_t)b], qt, kt);
+}
+
+fa_status_t fa_split_queries(const fa_desc_t* desc, const int64_t* actual_seq_qlen,
+                             const int64_t* actual_seq_kvlen, int32_t n_parts,
+                             const int64_t* cuts, int32_t part, fa_split_part_t* out,
+                             int64_t* out_seq_qlen, int64_t* out_seq_kvlen) {
+  clear_error();
+  return split_queries(desc, actual_seq_qlen, actual_seq_kvlen, n_parts, cuts, part, out,
+                       out_seq_qlen, out_seq_kvlen);
 }
 
 fa_status_t fa_plan_stats(const fa_desc_t* desc, const int64_t* prefix,
