@@ -563,17 +563,26 @@ __device__ void mma_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t
 }
 
 // Scores of this thread's row (128 keys of S_s) with the element mask of a
-// boundary tile applied (-inf where the key is not visible).
+// boundary tile applied (-inf where the key is not visible). The visible
+// columns [c_lo, c_hi] are tested as one unsigned range compare per element;
+// dense-mask bits (modes 0/1) are applied only when present.
 __device__ __forceinline__ void load_scores(uint32_t tS, float (&x)[128], bool partial, int c_lo,
-                                            int c_hi, const uint32_t (&mbits)[4]) {
+                                            int c_hi, bool dense, const uint32_t (&mbits)[4]) {
   uint32_t sv[128];
   tmem_ld128_wait(tS, sv);
 #pragma unroll
   for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sv[c]);
   if (partial) {
+    int lo = c_lo, width = c_hi - c_lo;
+    if (width < 0) lo = 1 << 20, width = 0;  // nothing visible
 #pragma unroll
     for (int c = 0; c < 128; ++c)
-      if (c < c_lo || c > c_hi || ((mbits[c >> 5] >> (c & 31)) & 1u)) x[c] = -INFINITY;
+      x[c] = ((unsigned)(c - lo) <= (unsigned)width) ? x[c] : -INFINITY;
+    if (dense) {
+#pragma unroll
+      for (int c = 0; c < 128; ++c)
+        x[c] = ((mbits[c >> 5] >> (c & 31)) & 1u) ? -INFINITY : x[c];
+    }
   }
 }
 
@@ -678,7 +687,7 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint
       }
       tc_fence_after();
       float x[128];
-      load_scores(tS, x, partial, c_lo, c_hi, mbits);
+      load_scores(tS, x, partial, c_lo, c_hi, mrow != nullptr, mbits);
       const float m_new = row_max128(x) * scale_log2;
       const bool resc = m_new > m_used + kRescaleLog2;
       float alpha = 1.f;
