@@ -10,16 +10,21 @@
 // One persistent CTA per SM, 16 warps, warp-specialised:
 //   warps 0-3   softmax of query sub-tile 0 (rows 0..127 of the item)
 //   warps 4-7   softmax of query sub-tile 1 (rows 128..255)
-//   warp 12     tcgen05.mma issuer (one thread; owns TMEM)
+//   warps 8-11  epilogue: O / l of both sub-tiles to global memory
+//   warp 12     S = Q K^T issuer (one thread; owns TMEM)
 //   warp 13     TMA producer (one thread)
-//   other warps idle (they give their registers to the softmax warps)
-// Tensor memory (512 columns): S0 | S1 | O0 | O1. S_s holds the fp32 scores
-// of sub-tile s; the softmax overwrites its first 64 columns with P (bf16
-// pairs), which feeds the P.V MMA directly from TMEM. O_s accumulates fp32.
-// MMA issue order per key tile t:  PV0(t), QK0(t+1), PV1(t), QK1(t+1), so
-// each softmax warpgroup has the time of two MMA groups to turn S into P,
-// and every S_s(t+1) commit also proves PV_s(t) complete (commits track all
-// earlier MMAs), which is what lets the softmax rescale O_s in place.
+//   warp 14     O += P V issuer (one thread)
+//   warp 15     idle
+// Tensor memory (512 columns): S0 | S1 | O0 | O1 (fp32 scores and output
+// accumulators of the two sub-tiles). P = exp(S - m) in bf16 goes to its own
+// buffer (shared memory at D = 128, free tensor memory columns at D = 64), so
+// the softmax releases S_s as soon as it has read it and the next QK of the
+// sub-tile runs while the softmax exponentiates.
+// The two MMA streams are issued by two threads, so that one thread's
+// barrier waits and commits (each of which stalls the tensor pipe while the
+// issuing thread handles it) overlap the other thread's MMAs. The softmax
+// waits for PV_s(t-1) before it overwrites the P buffer and before it
+// rescales O_s in place; the epilogue waits for the item's last PV.
 // Every mbarrier wait is bounded (globaltimer); on expiry the CTA records
 // the site in the error word, drains its in-flight copies and MMAs, frees
 // its tensor memory and exits.
@@ -39,21 +44,22 @@ namespace dev {
 constexpr int kThreads = 512;
 constexpr int kWarpMma = 12;
 constexpr int kWarpLoad = 13;
+constexpr int kWarpPv = 14;
 // Register split (setmaxnreg) over the 512 x 128 registers of the launch:
-// softmax warpgroups 0-1 take 208, the idle warpgroup 2 keeps 24, the
-// warpgroup of the MMA and TMA warps keeps 72.
-constexpr int kRegsSoftmax = 208;
-constexpr int kRegsIdle = 24;
-constexpr int kRegsControl = 72;
-constexpr int kRegsTotal = 2 * 128 * kRegsSoftmax + 128 * kRegsIdle + 128 * kRegsControl;
+// softmax warpgroups 0-1 take 192, the epilogue warpgroup 2 and the
+// warpgroup of the MMA and TMA warps keep 64 each.
+constexpr int kRegsSoftmax = 192;
+constexpr int kRegsEpi = 64;
+constexpr int kRegsControl = 64;
+constexpr int kRegsTotal = 2 * 128 * kRegsSoftmax + 128 * kRegsEpi + 128 * kRegsControl;
 static_assert(kRegsTotal == kThreads * 128, "register split must equal the launch allocation");
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
-constexpr int kPChunks = 4;           // P is exponentiated and stored 32 keys at a time
 
 // Where a wait gave up (error word bits 8..15).
 enum WaitSite : uint32_t {
   kSiteQEmpty = 1, kSiteKvEmpty = 2, kSiteQFull = 3, kSiteKvFull = 4, kSitePFull = 5,
-  kSiteSFull = 6, kSiteODone = 7, kSiteDrain = 8,
+  kSiteSFull = 6, kSiteOPv = 7, kSiteDrain = 8, kSiteSFree = 9, kSiteOFree = 10,
+  kSiteMufu = 11, kSiteEpi = 12, kSiteStatFree = 13,
 };
 
 template <int D>
@@ -61,24 +67,42 @@ struct Cfg {
   static constexpr int kChunks = D / 64;                 // 64-column (128-byte) chunks per row
   static constexpr uint32_t kChunkBytes = 128u * 128u;   // 128 rows x 128 bytes
   static constexpr uint32_t kTileBytes = 128u * D * 2u;  // 128 rows of Q, K or V
-  static constexpr int kStages = (D == 128) ? 4 : 8;     // K/V ring depth
+  // P = exp(S - m) in bf16 feeds the P.V MMA from shared memory at D = 128
+  // (tensor memory is full with S0 | S1 | O0 | O1) and from its own tensor
+  // memory columns at D = 64.
+  static constexpr bool kPInTmem = (D == 64);
+  static constexpr int kStages = (D == 128) ? 3 : 8;     // K/V ring depth
   static constexpr uint32_t kQBytes = 2u * kTileBytes;
   static constexpr uint32_t kKVBytes = kStages * kTileBytes;
-  static constexpr uint32_t kCtlBytes = 512u;
-  static constexpr uint32_t kSmemBytes = 1024u + kQBytes + kKVBytes + kCtlBytes;
+  static constexpr uint32_t kPTileBytes = 128u * 128u * 2u;  // P of one sub-tile (bf16)
+  static constexpr uint32_t kPBytes = kPInTmem ? 0u : 2u * kPTileBytes;
+  static constexpr uint32_t kCtlBytes = 1024u;   // barriers
+  static constexpr uint32_t kStatBytes = 1024u;  // 1/l of the 2 x 128 rows
+  static constexpr uint32_t kSmemBytes =
+      1024u + kQBytes + kKVBytes + kPBytes + kCtlBytes + kStatBytes;
   static constexpr uint32_t kTmemCols = 512u;
-  // TMEM columns of S_s / P_s and of O_s
+  // TMEM columns of S_s and of O_s
   __host__ __device__ static constexpr uint32_t col_s(int s) { return s ? 128u : 0u; }
   __host__ __device__ static constexpr uint32_t col_o(int s) { return s ? 256u + D : 256u; }
+  // TMEM columns of P_s when kPInTmem (64 columns of bf16 pairs each)
+  __host__ __device__ static constexpr uint32_t col_p(int s) { return 256u + 2u * D + 64u * s; }
+  static_assert(!kPInTmem || 256u + 2u * D + 128u <= kTmemCols, "tensor memory budget");
   static_assert(kSmemBytes <= 227u * 1024u, "shared memory budget");
 };
 
 template <int NS>
 struct Ctl {
-  uint64_t q_full, q_empty;
+  uint64_t q_full[2], q_empty[2];  // Q sub-tile s loaded / no longer read
   uint64_t kv_full[NS], kv_empty[NS];
-  uint64_t s_full[2], p_full[2], o_done[2];
-  uint64_t drain[1];
+  uint64_t s_full[2];  // S_s in TMEM
+  uint64_t s_free[2];  // S_s read into registers: the next QK_s may overwrite it
+  uint64_t p_full[2];  // P_s in shared memory
+  uint64_t o_pv[2];    // one PV_s finished (O_s updated, P_s buffer free again)
+  uint64_t mufu[2];      // turn of softmax warpgroup s on the exponential unit
+  uint64_t epi_full[2];   // 1/l of sub-tile s written for the epilogue (every item)
+  uint64_t stat_free[2];  // epilogue has read that 1/l (every item)
+  uint64_t o_free[2];     // epilogue has read O_s (items that visit a key tile)
+  uint64_t drain[2];  // one per MMA-issuing thread
   uint32_t tmem_base;
   volatile int abort_flag;
 };
@@ -182,34 +206,6 @@ __device__ __forceinline__ float row_max128(const float (&x)[128]) {
   return max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
-// x <- 2^(x * scale_log2 - ref) in place; returns the row sum (eight
-// independent partial sums). kPoly: some columns use ex2_poly_x2.
-template <bool kPoly>
-__device__ __forceinline__ float exp_rows(float (&x)[128], float scale_log2, float ref) {
-  const uint64_t m2 = pack_f32x2(scale_log2, scale_log2);
-  const uint64_t c2 = pack_f32x2(-ref, -ref);
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int c = 0; c < 128; c += 2) {
-    float a = x[c], b = x[c + 1];
-    fma_x2(a, b, m2, c2);
-    if (kPoly && (c & 7) < kPolyPer8) {
-      ex2_poly_x2(a, b);
-    } else {
-      a = ex2(a);
-      b = ex2(b);
-    }
-    x[c] = a;
-    x[c + 1] = b;
-    const int k = (c >> 1) & 3;
-    add_x2(acc[2 * k], acc[2 * k + 1], a, b);
-  }
-  add_x2(acc[0], acc[1], acc[2], acc[3]);
-  add_x2(acc[4], acc[5], acc[6], acc[7]);
-  add_x2(acc[0], acc[1], acc[4], acc[5]);
-  return acc[0] + acc[1];
-}
-
 // ----------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -265,6 +261,53 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, con
       }
     }
   }
+}
+
+// Turn token on the exponential unit (no data is handed over, so there is no
+// memory clobber: the score registers stay in registers across the wait).
+// Returns the warp-wide result and a 0.f that the caller adds into the
+// exponent offset, so no exponential can be scheduled ahead of the wait;
+// `dep` (the row maximum) is an input of the first poll, so the work that
+// produces it cannot sink into the turn either.
+__device__ __forceinline__ bool mbar_try_wait_token(uint64_t* bar, uint32_t parity, float dep) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity), "f"(dep));
+  return done != 0;
+}
+
+__device__ __forceinline__ bool wait_token(uint64_t* bar, uint32_t parity, const WaitCtx& w,
+                                           float dep, float& zero) {
+  bool ok = mbar_try_wait_token(bar, parity, dep);
+  if (!ok) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+      if (mbar_try_wait_token(bar, parity, dep)) {
+        ok = true;
+        break;
+      }
+      if ((spin & 63u) == 0u) {
+        if (*w.abort_flag) break;
+        if (globaltimer_ns() - t0 > w.timeout_ns) {
+          *w.abort_flag = 1;
+          atomicOr(w.err_word, kErrTimeout | (kSiteMufu << kErrWhereShift));
+          break;
+        }
+      }
+    }
+  }
+  asm volatile("mov.b32 %0, 0f00000000;" : "=f"(zero));
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Hands the exponential unit to the other warpgroup once `dep` (a value
+// computed from every exponential of this turn) exists.
+__device__ __forceinline__ void arrive_token(uint64_t* bar, float dep) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)), "f"(dep));
 }
 
 // Whole-warp wait: every lane waits, the warp proceeds only if all did.
@@ -379,13 +422,54 @@ __device__ __forceinline__ bool active(const TileRange& t, int j) { return j >= 
 
 // ----------------------------------------------------------------- roles
 
+// TMA producer (one thread). The ring carries K and V tiles in exactly the
+// order the MMA warp consumes them: K(t+1) ahead of V(t) (the scores of tile
+// t+1 are computed before P(t) is multiplied by V(t)), and an item's first K
+// ahead of the previous item's last V. Per item: Q of sub-tile 0, the first
+// K tile, Q of sub-tile 1, the previous item's last V, then K(t+1), V(t)
+// for the item's key tiles but the last, whose V waits for the next item's
+// first K (or the end of the work list). A Q tile is loaded once its buffer
+// is released by the last QK of the previous item on that sub-tile; placing
+// Q1 after the first K keeps a late Q1 release from holding back K.
 template <int D>
 __device__ void load_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint8_t* sQ,
                           uint8_t* sKV, const WaitCtx& w) {
   using C = Cfg<D>;
   constexpr int NS = C::kStages;
-  uint32_t ring = 0, q_loads = 0;
+  uint32_t ring = 0;
+  uint32_t nq[2] = {0u, 0u};
   bool ok = true;
+  auto load_q = [&](const WorkItem& it, const SeqRec& sr, int st, int bc) -> bool {
+    if (nq[st] > 0 && !wait_bounded(&ctl->q_empty[st], (nq[st] - 1) & 1u, w, kSiteQEmpty))
+      return false;
+    const bool drop = (p.debug_flags & kDebugDropFirstQ) && blockIdx.x == 0 && nq[0] + nq[1] == 0;
+    if (!drop) {
+      mbar_expect_tx(&ctl->q_full[st], C::kTileBytes);
+      const int row = sr.q_off + it.qblk * kBlockM + st * kTileM;
+#pragma unroll
+      for (int c = 0; c < C::kChunks; ++c)
+        tma_load_4d(sQ + st * C::kTileBytes + c * C::kChunkBytes, &p.tm_q, &ctl->q_full[st],
+                    c * 64, row, it.h, bc);
+    }
+    ++nq[st];
+    return true;
+  };
+  auto load_kv = [&](const CUtensorMap* tm, int row, int h, int bc) -> bool {
+    const uint32_t st = ring % NS;
+    if (ring >= (uint32_t)NS &&
+        !wait_bounded(&ctl->kv_empty[st], ((ring / NS) - 1) & 1u, w, kSiteKvEmpty))
+      return false;
+    mbar_expect_tx(&ctl->kv_full[st], C::kTileBytes);
+#pragma unroll
+    for (int c = 0; c < C::kChunks; ++c)
+      tma_load_4d(sKV + st * C::kTileBytes + c * C::kChunkBytes, tm, &ctl->kv_full[st], c * 64,
+                  row, h, bc);
+    ++ring;
+    return true;
+  };
+  struct PendingV {
+    int row, h, bc;
+  } pend{0, -1, 0};
   for (int k = 0; ok; ++k) {
     const int idx = item_index(k);
     if (idx >= p.n_items) break;
@@ -394,48 +478,26 @@ __device__ void load_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint8_t
     const ItemPlan ip = plan_item(sr, it.qblk);
     if (ip.hi <= ip.lo) continue;
     const int bc = p.tnd ? 0 : it.b;
-    if (q_loads > 0 && !wait_bounded(&ctl->q_empty, (q_loads - 1) & 1u, w, kSiteQEmpty)) {
-      ok = false;
-      break;
+    if (ip.tr[0].hi > ip.tr[0].lo) ok = load_q(it, sr, 0, bc);
+    if (ok) ok = load_kv(&p.tm_k, sr.kv_off + ip.lo * kTileN, it.h, bc);
+    if (ok && ip.tr[1].hi > ip.tr[1].lo) ok = load_q(it, sr, 1, bc);
+    // The previous item's last V follows this item's first K: the MMA warp
+    // computes those scores before it finishes the previous item.
+    if (ok && pend.h >= 0) ok = load_kv(&p.tm_v, pend.row, pend.h, pend.bc);
+    for (int t = ip.lo; t + 1 < ip.hi && ok; ++t) {
+      ok = load_kv(&p.tm_k, sr.kv_off + (t + 1) * kTileN, it.h, bc);
+      if (ok) ok = load_kv(&p.tm_v, sr.kv_off + t * kTileN, it.h, bc);
     }
-    const bool drop = (p.debug_flags & kDebugDropFirstQ) && blockIdx.x == 0 && q_loads == 0;
-    if (!drop) {
-      mbar_expect_tx(&ctl->q_full, ip.nsub * C::kTileBytes);
-      for (int st = 0; st < ip.nsub; ++st) {
-        const int row = sr.q_off + it.qblk * kBlockM + st * kTileM;
-#pragma unroll
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sQ + st * C::kTileBytes + c * C::kChunkBytes, &p.tm_q, &ctl->q_full, c * 64,
-                      row, it.h, bc);
-      }
-    }
-    ++q_loads;
-    for (int t = ip.lo; t < ip.hi && ok; ++t) {
-#pragma unroll 1
-      for (int kv = 0; kv < 2; ++kv) {
-        const uint32_t st = ring % NS;
-        if (ring >= (uint32_t)NS &&
-            !wait_bounded(&ctl->kv_empty[st], ((ring / NS) - 1) & 1u, w, kSiteKvEmpty)) {
-          ok = false;
-          break;
-        }
-        mbar_expect_tx(&ctl->kv_full[st], C::kTileBytes);
-        const CUtensorMap* tm = kv == 0 ? &p.tm_k : &p.tm_v;
-        const int row = sr.kv_off + t * kTileN;
-#pragma unroll
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sKV + st * C::kTileBytes + c * C::kChunkBytes, tm, &ctl->kv_full[st],
-                      c * 64, row, it.h, bc);
-        ++ring;
-      }
-    }
+    pend = PendingV{sr.kv_off + (ip.hi - 1) * kTileN, it.h, bc};
   }
+  if (ok && pend.h >= 0) ok = load_kv(&p.tm_v, pend.row, pend.h, pend.bc);
   if (!ok) {
     // Abort: let every copy this thread started land before the CTA exits.
     const uint32_t first = ring > (uint32_t)NS ? ring - NS : 0u;
     for (uint32_t r = first; r < ring; ++r)
       wait_bounded(&ctl->kv_full[r % NS], (r / NS) & 1u, w, kSiteDrain, false);
-    if (q_loads > 0) wait_bounded(&ctl->q_full, (q_loads - 1) & 1u, w, kSiteDrain, false);
+    for (int st = 0; st < 2; ++st)
+      if (nq[st] > 0) wait_bounded(&ctl->q_full[st], (nq[st] - 1) & 1u, w, kSiteDrain, false);
   }
 }
 
@@ -457,109 +519,188 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem, const uint8_t* sQ, const
 }
 
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t tmem, const uint8_t* sKV, int sub, uint32_t vst,
-                                         bool accumulate) {
+__device__ __forceinline__ void issue_pv(uint32_t tmem, const uint8_t* sP, const uint8_t* sKV,
+                                         int sub, uint32_t vst, bool accumulate) {
   using C = Cfg<D>;
   constexpr uint32_t idesc = idesc_bf16(128, D, true);
   // V is MN-major (D contiguous): step k moves 16 key rows = 2048 bytes.
   const uint64_t b0 = sdesc(smem_u32(sKV) + vst * C::kTileBytes, C::kChunkBytes, 1024u);
-  const uint32_t a = tmem + C::col_s(sub);  // P: 128 bf16 = 64 columns
   const uint32_t d = tmem + C::col_o(sub);
+  if constexpr (C::kPInTmem) {
+    // P in tensor memory: 16 keys = 8 columns of bf16 pairs per step.
+    const uint32_t a = tmem + C::col_p(sub);
 #pragma unroll
-  for (int k = 0; k < kTileN / 16; ++k)
-    mma_ts(d, a + k * 8u, b0 + (uint64_t)(k * (2048u >> 4)), idesc,
-           (accumulate || k > 0) ? 1u : 0u);
+    for (int k = 0; k < kTileN / 16; ++k)
+      mma_ts(d, a + k * 8u, b0 + (uint64_t)(k * (2048u >> 4)), idesc,
+             (accumulate || k > 0) ? 1u : 0u);
+  } else {
+    // P in shared memory, K-major like Q: step k advances 32 bytes in a
+    // 128-byte row, every 4 steps the next 64-key chunk.
+    const uint64_t a0 = sdesc(smem_u32(sP) + sub * C::kPTileBytes, 16u, 1024u);
+#pragma unroll
+    for (int k = 0; k < kTileN / 16; ++k) {
+      const uint64_t a_off = (uint64_t)(((k >> 2) * C::kChunkBytes + (k & 3) * 32u) >> 4);
+      mma_ss(d, a0 + a_off, b0 + (uint64_t)(k * (2048u >> 4)), idesc,
+             (accumulate || k > 0) ? 1u : 0u);
+    }
+  }
 }
 
-// MMA issue (one thread). Per key tile t, in this order:
-//   O_0 += P_0(t) V(t); S_0(t+1) = Q_0 K(t+1)^T; O_1 += P_1(t) V(t);
-//   S_1(t+1) = Q_1 K(t+1)^T
-// so each softmax warpgroup has two MMA groups' time to turn S into P. Both
-// ring waits come before the first group and the commits follow the QK
-// groups, so consecutive groups go out with only the P wait between them:
-// the tensor pipe queues few instructions and any gap in issue idles it.
+// Key-tile ranges of an item as the MMA warps need them: sub-tile s visits
+// [lo[s], hi[s]), the item visits [lo[2], hi[2]); `pos` is the item's
+// position in this CTA's list.
+struct MmaPlan {
+  int lo[3], hi[3];
+  int pos;
+};
+
+// Next item of this CTA with at least one key tile, from position k on.
+__device__ __forceinline__ bool next_item(const FwdParams& p, int& k, MmaPlan& mp) {
+  for (;; ++k) {
+    const int idx = item_index(k);
+    if (idx >= p.n_items) return false;
+    const WorkItem it = p.items[idx];
+    const ItemPlan ip = plan_item(p.seqs[it.b], it.qblk);
+    if (ip.hi > ip.lo) {
+      mp.pos = k;
+      ++k;
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        mp.lo[s] = ip.tr[s].lo;
+        mp.hi[s] = ip.tr[s].hi;
+      }
+      mp.lo[2] = ip.lo;
+      mp.hi[2] = ip.hi;
+      return true;
+    }
+  }
+}
+
+__device__ __forceinline__ bool act(const MmaPlan& mp, int s, int t) {
+  return t >= mp.lo[s] && t < mp.hi[s];
+}
+
+// Ring position of the K and V tiles of the g-th key tile this CTA visits
+// (counted over its items in order). The TMA producer loads K(g+1) ahead of
+// V(g): K(0), K(1), V(0), K(2), V(1), ..., K(last), V(last-1), V(last).
+__device__ __forceinline__ uint32_t ring_k(uint32_t g) { return g == 0 ? 0u : 2u * g - 1u; }
+__device__ __forceinline__ uint32_t ring_v(uint32_t g, bool last) {
+  return last ? 2u * g + 1u : 2u * g + 2u;
+}
+
+// S = Q K^T issue (one thread). Walks the CTA's key tiles in order; for each
+// tile t of an item and each sub-tile s that visits it, waits until the
+// softmax has read S_s of the previous tile and issues S_s = Q_s K(t)^T.
+// It runs ahead of the P.V stream (another thread), limited only by the
+// softmax releasing S, so the scores of the next tile, also across item
+// boundaries, are ready when the softmax wants them.
 template <int D>
-__device__ void mma_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t tmem,
-                         const uint8_t* sQ, const uint8_t* sKV, const WaitCtx& w) {
+__device__ void qk_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t tmem,
+                        const uint8_t* sQ, const uint8_t* sKV, const WaitCtx& w) {
   using C = Cfg<D>;
   constexpr int NS = C::kStages;
-  uint32_t ring = 0, q_loads = 0;
-  uint32_t p_count[2] = {0u, 0u};
+  uint32_t g = 0;                  // key tiles visited so far
+  uint32_t nq[2] = {0u, 0u};       // Q loads awaited per sub-tile
+  uint32_t n_qk[2] = {0u, 0u};     // QK MMAs issued per sub-tile
   bool ok = true;
-  for (int k = 0; ok; ++k) {
-    const int idx = item_index(k);
-    if (idx >= p.n_items) break;
-    const WorkItem it = p.items[idx];
-    const SeqRec sr = p.seqs[it.b];
-    const ItemPlan ip = plan_item(sr, it.qblk);
-    if (ip.hi <= ip.lo) continue;
-    if (!wait_bounded(&ctl->q_full, q_loads & 1u, w, kSiteQFull)) {
-      ok = false;
-      break;
-    }
-    ++q_loads;
-    uint32_t kst = ring % NS;
-    if (!wait_bounded(&ctl->kv_full[kst], (ring / NS) & 1u, w, kSiteKvFull)) {
-      ok = false;
-      break;
-    }
-    ++ring;
-#pragma unroll
-    for (int s = 0; s < 2; ++s)
-      if (active(ip.tr[s], ip.lo)) {
-        issue_qk<D>(tmem, sQ, sKV, s, kst);
-        mma_commit(&ctl->s_full[s]);
-      }
-    mma_commit(&ctl->kv_empty[kst]);
-    if (ip.lo + 1 == ip.hi) mma_commit(&ctl->q_empty);
-    bool first[2] = {true, true};
-    for (int t = ip.lo; t < ip.hi && ok; ++t) {
-      const uint32_t vst = ring % NS;
-      if (!wait_bounded(&ctl->kv_full[vst], (ring / NS) & 1u, w, kSiteKvFull)) {
+  int k = 0;
+  MmaPlan cur;
+  while (ok && next_item(p, k, cur)) {
+    bool q_ready[2] = {false, false};
+    for (int t = cur.lo[2]; t < cur.hi[2] && ok; ++t, ++g) {
+      const uint32_t r = ring_k(g);
+      if (!wait_bounded(&ctl->kv_full[r % NS], (r / NS) & 1u, w, kSiteKvFull)) {
         ok = false;
         break;
       }
-      ++ring;
-      const bool nxt = t + 1 < ip.hi;
-      if (nxt) {
-        kst = ring % NS;
-        if (!wait_bounded(&ctl->kv_full[kst], (ring / NS) & 1u, w, kSiteKvFull)) {
-          ok = false;
-          break;
-        }
-        ++ring;
-      }
 #pragma unroll
       for (int s = 0; s < 2; ++s) {
-        if (active(ip.tr[s], t)) {
-          if (!wait_bounded(&ctl->p_full[s], p_count[s] & 1u, w, kSitePFull)) {
+        if (!act(cur, s, t)) continue;
+        if (!q_ready[s]) {
+          if (!wait_bounded(&ctl->q_full[s], nq[s] & 1u, w, kSiteQFull)) {
             ok = false;
             break;
           }
-          ++p_count[s];
-          tc_fence_after();
-          issue_pv<D>(tmem, sKV, s, vst, !first[s]);
-          first[s] = false;
-          if (t == ip.tr[s].hi - 1) mma_commit(&ctl->o_done[s]);
+          ++nq[s];
+          q_ready[s] = true;
         }
-        if (nxt && active(ip.tr[s], t + 1)) {
-          issue_qk<D>(tmem, sQ, sKV, s, kst);
-          mma_commit(&ctl->s_full[s]);
+        if (n_qk[s] > 0 &&
+            !wait_bounded(&ctl->s_free[s], (n_qk[s] - 1) & 1u, w, kSiteSFree)) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        issue_qk<D>(tmem, sQ, sKV, s, r % NS);
+        mma_commit(&ctl->s_full[s]);
+        ++n_qk[s];
+        if (t == cur.hi[s] - 1) mma_commit(&ctl->q_empty[s]);  // last read of this Q
       }
-      if (!ok) break;
-      mma_commit(&ctl->kv_empty[vst]);
-      if (nxt) {
-        mma_commit(&ctl->kv_empty[kst]);
-        if (t + 2 == ip.hi) mma_commit(&ctl->q_empty);
-      }
+      if (ok) mma_commit(&ctl->kv_empty[r % NS]);
     }
   }
-  if (!ok) {
-    // Abort: wait until every MMA issued so far has finished with TMEM/SMEM.
-    mma_commit(&ctl->drain[0]);
-    wait_bounded(&ctl->drain[0], 0u, w, kSiteDrain, false);
+  // Wait until every MMA this thread issued (and its commits) has finished
+  // with tensor and shared memory.
+  mma_commit(&ctl->drain[0]);
+  wait_bounded(&ctl->drain[0], 0u, w, kSiteDrain, false);
+}
+
+// O += P V issue (one thread). For each key tile t and each sub-tile that
+// visits it, waits for P_s(t) from the softmax and issues O_s += P_s V(t);
+// the commit after it tells the softmax that O_s is updated and that the P
+// buffer may be rewritten. The first PV of an item overwrites O_s, so it
+// waits until the epilogue has read O_s of the previous item that had one.
+template <int D>
+__device__ void pv_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t tmem,
+                        const uint8_t* sP, const uint8_t* sKV, const WaitCtx& w) {
+  using C = Cfg<D>;
+  constexpr int NS = C::kStages;
+  uint32_t g = 0;
+  uint32_t p_count[2] = {0u, 0u};  // P tiles consumed per sub-tile
+  uint32_t n_act[2] = {0u, 0u};    // items so far in which sub-tile s visits a key tile
+  bool ok = true;
+  int k = 0;
+  MmaPlan cur;
+  bool have = next_item(p, k, cur);
+  while (ok && have) {
+    MmaPlan nxt;
+    const bool have_next = next_item(p, k, nxt);
+    bool first[2] = {true, true};
+    for (int t = cur.lo[2]; t < cur.hi[2] && ok; ++t, ++g) {
+      const uint32_t r = ring_v(g, !have_next && t + 1 == cur.hi[2]);
+      if (!wait_bounded(&ctl->kv_full[r % NS], (r / NS) & 1u, w, kSiteKvFull)) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        if (!act(cur, s, t)) continue;
+        if (!wait_bounded(&ctl->p_full[s], p_count[s] & 1u, w, kSitePFull)) {
+          ok = false;
+          break;
+        }
+        ++p_count[s];
+        // o_free[s] completes one phase per item that visits a key tile of
+        // sub-tile s: wait for the one of the previous such item.
+        if (first[s]) {
+          if (n_act[s] > 0 &&
+              !wait_bounded(&ctl->o_free[s], (n_act[s] - 1) & 1u, w, kSiteOFree)) {
+            ok = false;
+            break;
+          }
+          ++n_act[s];
+        }
+        tc_fence_after();
+        issue_pv<D>(tmem, sP, sKV, s, r % NS, !first[s]);
+        first[s] = false;
+        mma_commit(&ctl->o_pv[s]);
+      }
+      if (ok) mma_commit(&ctl->kv_empty[r % NS]);
+    }
+    cur = nxt;
+    have = have_next;
   }
+  mma_commit(&ctl->drain[1]);
+  wait_bounded(&ctl->drain[1], 0u, w, kSiteDrain, false);
 }
 
 // Scores of this thread's row (128 keys of S_s) with the element mask of a
@@ -586,14 +727,17 @@ __device__ __forceinline__ void load_scores(uint32_t tS, float (&x)[128], bool p
   }
 }
 
-// Exponentiate keys [32 c, 32 c + 32) of the row against `ref`, add them to
-// the eight partial sums and pack P into 16 bf16 pairs.
+// x <- 2^(x * scale_log2 - ref) for the 128 keys of the row, packed into 64
+// bf16 pairs (even key in the low half); returns the row sum of the fp32
+// values (eight independent partial sums).
 template <bool kPoly>
-__device__ __forceinline__ void exp_chunk(float (&x)[128], int chunk, uint64_t m2, uint64_t c2,
-                                          float (&acc)[8], uint32_t (&pk)[16]) {
+__device__ __forceinline__ float exp_pack(const float (&x)[128], float scale_log2, float ref,
+                                          uint32_t (&pk)[64]) {
+  const uint64_t m2 = pack_f32x2(scale_log2, scale_log2);
+  const uint64_t c2 = pack_f32x2(-ref, -ref);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int j = 0; j < 32; j += 2) {
-    const int c = chunk * 32 + j;
+  for (int c = 0; c < 128; c += 2) {
     float a = x[c], b = x[c + 1];
     fma_x2(a, b, m2, c2);
     if (kPoly && (c & 7) < kPolyPer8) {
@@ -602,54 +746,78 @@ __device__ __forceinline__ void exp_chunk(float (&x)[128], int chunk, uint64_t m
       a = ex2(a);
       b = ex2(b);
     }
-    const int k = (j >> 1) & 3;
+    const int k = (c >> 1) & 3;
     add_x2(acc[2 * k], acc[2 * k + 1], a, b);
-    pk[j >> 1] = pack_bf16(a, b);
+    pk[c >> 1] = pack_bf16(a, b);
   }
-}
-
-// Exponentiate the row chunk by chunk, storing each chunk of P as soon as it
-// is packed; one arrival on p_full once every store has landed.
-template <bool kPoly>
-__device__ __forceinline__ float exp_store_p(float (&x)[128], float scale_log2, float ref,
-                                             uint32_t tS, uint64_t* p_full) {
-  const uint64_t m2 = pack_f32x2(scale_log2, scale_log2);
-  const uint64_t c2 = pack_f32x2(-ref, -ref);
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int c = 0; c < kPChunks; ++c) {
-    uint32_t pk[16];
-    exp_chunk<kPoly>(x, c, m2, c2, acc, pk);
-    tmem_st16(tS + 16u * c, pk);
-  }
-  tmem_st_wait();
-  tc_fence_before();
-  mbar_arrive(p_full);
   add_x2(acc[0], acc[1], acc[2], acc[3]);
   add_x2(acc[4], acc[5], acc[6], acc[7]);
   add_x2(acc[0], acc[1], acc[4], acc[5]);
   return acc[0] + acc[1];
 }
 
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// Row `row` of a 128 x 128 bf16 P tile at `base` (1024-byte aligned), in the
+// layout a TMA load with 128-byte swizzle gives a 64-column box and the MMA
+// reads as K-major: two 64-key chunks of 16 KB, rows 128 bytes apart, and
+// the 16-byte unit u of row r at unit position u ^ (r % 8). Eight
+// consecutive rows cover all 32 banks, so every store is conflict-free.
+__device__ __forceinline__ void store_p_smem(uint32_t base, int row, const uint32_t (&pk)[64]) {
+  const uint32_t rb = base + (uint32_t)row * 128u;
+  const uint32_t sw = (uint32_t)row & 7u;
+#pragma unroll
+  for (int u = 0; u < 16; ++u)
+    st_shared_v4(rb + (uint32_t)(u >> 3) * 16384u + ((((uint32_t)u & 7u) ^ sw) << 4),
+                 pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the
+// tensor core's (async-proxy) reads that follow the next barrier.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Softmax of query sub-tile `sub` (one warpgroup, one row per thread). Per
+// key tile: read S_s, release it to the next QK, row maximum, then - in
+// strict alternation with the other softmax warpgroup, so that the two
+// never compete for the exponential unit - exponentiate and pack P; then
+// wait for the previous PV (it still reads the P buffer and O_s must hold
+// it before a rescale), rescale O_s if the reference maximum moved, store P.
+// Every tile of the item's union range is one turn for both warpgroups; a
+// warpgroup that does not visit the tile passes its turn on. At the end of
+// an item it writes the row's log-sum-exp and hands 1/l to the epilogue
+// warpgroup.
 template <int D>
-__device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t tmem,
-                             int sub, const WaitCtx& w) {
+__device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, float* inv_l_sm,
+                             uint32_t tmem, uint8_t* sP, int sub, const WaitCtx& w) {
   using C = Cfg<D>;
   const int wq = (threadIdx.x >> 5) & 3;           // TMEM lane quarter of this warp
-  const int row = wq * 32 + (threadIdx.x & 31);    // row of the sub-tile = TMEM lane
+  const int lane = threadIdx.x & 31;
+  const int row = wq * 32 + lane;                  // row of the sub-tile = TMEM lane
   const uint32_t lane_bits = (uint32_t)(wq * 32) << 16;
   const uint32_t tS = tmem + lane_bits + C::col_s(sub);
   const uint32_t tO = tmem + lane_bits + C::col_o(sub);
+  const uint32_t tP = tmem + lane_bits + C::col_p(sub);
+  const uint32_t sPs = smem_u32(sP) + sub * C::kPTileBytes;
   const float scale_log2 = p.scale_log2;
-  uint32_t s_count = 0, o_count = 0;
+  uint32_t s_count = 0;   // S tiles consumed
+  uint32_t pv_count = 0;  // P tiles produced = PV MMAs of this sub-tile
+  uint32_t turn = 0;      // exponential-unit turns taken
   bool ok = true;
   for (int k = 0; ok; ++k) {
     const int idx = item_index(k);
     if (idx >= p.n_items) break;
     const WorkItem it = p.items[idx];
     const SeqRec sr = p.seqs[it.b];
+    const ItemPlan ip = plan_item(sr, it.qblk);
+    const TileRange tr = ip.tr[sub];
     const int64_t r0 = (int64_t)it.qblk * kBlockM + sub * kTileM;
-    const TileRange tr = tile_range(sr, r0);
     const int i = (int)(r0 + row);  // query row inside the sequence
     const bool row_valid = i < sr.sq;
     // Visible keys of this row: [jlo, jhi] (empty when jlo > jhi).
@@ -663,7 +831,23 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint
       mrow = p.mask + it.b * p.m_sb + it.h * p.m_sh + (int64_t)i * p.m_si;
     float m_used = -INFINITY;  // reference max (log2 units, scaled)
     float l = 0.f;             // running sum relative to m_used
-    for (int t = tr.lo; t < tr.hi; ++t) {
+    for (int t = ip.lo; t < ip.hi; ++t) {
+      // Turn on the exponential unit: warpgroup 0 goes first in every tile.
+      uint64_t* my_turn = &ctl->mufu[sub];
+      const uint32_t turn_par = (sub == 0 ? turn - 1 : turn) & 1u;
+      const bool first_turn = sub == 0 && turn == 0;
+      ++turn;
+      if (t < tr.lo || t >= tr.hi) {
+        // Not visited by this sub-tile: pass the turn on.
+        float zero = 0.f;
+        if (!first_turn && !wait_token(my_turn, turn_par, w, 0.f, zero)) {
+          ok = false;
+          break;
+        }
+        __syncwarp();
+        if (lane == 0) arrive_token(&ctl->mufu[sub ^ 1], zero);
+        continue;
+      }
       if (!wait_warp(&ctl->s_full[sub], s_count & 1u, w, kSiteSFull)) {
         ok = false;
         break;
@@ -688,6 +872,9 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint
       tc_fence_after();
       float x[128];
       load_scores(tS, x, partial, c_lo, c_hi, mrow != nullptr, mbits);
+      // S_s is in registers: the next QK of this sub-tile may overwrite it.
+      tc_fence_before();
+      mbar_arrive(&ctl->s_free[sub]);
       const float m_new = row_max128(x) * scale_log2;
       const bool resc = m_new > m_used + kRescaleLog2;
       float alpha = 1.f;
@@ -696,60 +883,123 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint
         l *= alpha;
         m_used = m_new;
       }
-      // O_s already holds PV(t-1) (the S_s(t) commit tracked it); rescale it
-      // in place when this row's reference max moved, before the first P
-      // chunk lets PV(t) accumulate. Not on the item's first tile: its PV
-      // overwrites O_s.
-      if (t > tr.lo && __any_sync(0xffffffffu, resc)) {
+      float zero = 0.f;
+      if (!first_turn && !wait_token(my_turn, turn_par, w, m_new, zero)) {
+        ok = false;
+        break;
+      }
+      const float ref = ((m_used == -INFINITY) ? 0.f : m_used) + zero;
+      uint32_t pk[64];
+      const float lsum = partial ? exp_pack<false>(x, scale_log2, ref, pk)
+                                 : exp_pack<true>(x, scale_log2, ref, pk);
+      l += lsum;
+      __syncwarp();
+      if (lane == 0) arrive_token(&ctl->mufu[sub ^ 1], lsum);
+      if (pv_count > 0) {
+        // The previous PV of this sub-tile must be done: it still reads the
+        // P buffer, and O_s must hold it before it is rescaled.
+        if (!wait_warp(&ctl->o_pv[sub], (pv_count - 1) & 1u, w, kSiteOPv)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // Not on the item's first tile: the first PV of an item overwrites O_s.
+        if (t > tr.lo && __any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t ov[32];
+            tmem_ld32_wait(tO + ch * 32u, ov);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+            tmem_st32(tO + ch * 32u, ov);
+          }
+        }
+      }
+      if constexpr (C::kPInTmem) {
+        tmem_st32(tP, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(tP + 32u, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+      } else {
+        store_p_smem(sPs, row, pk);
+        fence_proxy_async_smem();
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&ctl->p_full[sub]);
+      ++pv_count;
+    }
+    if (!ok) break;
+    // lse = ln(sum exp(scale q.k)); 1/l goes to the epilogue once it has
+    // taken the previous item's value.
+    if (k > 0 && !wait_warp(&ctl->stat_free[sub], (k - 1) & 1u, w, kSiteStatFree)) {
+      ok = false;
+      break;
+    }
+    inv_l_sm[sub * kTileM + row] = l > 0.f ? 1.f / l : 0.f;
+    mbar_arrive(&ctl->epi_full[sub]);
+    if (row_valid) {
+      const float lse = l > 0.f ? (m_used + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      p.lse[it.b * p.l_sb + it.h * p.l_sh + sr.q_off + i] = lse;
+    }
+  }
+}
+
+// Epilogue (one warpgroup, one row of each sub-tile per thread): for every
+// item and sub-tile, once the softmax has handed over 1/l and the item's last
+// PV is done, O_s / l -> bf16 rows in global memory (zeros for rows that see
+// no key); 1/l is released as soon as it is read, O_s once it is read.
+template <int D>
+__device__ void epilogue_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl,
+                              const float* inv_l_sm, uint32_t tmem, const WaitCtx& w) {
+  using C = Cfg<D>;
+  const int wq = (threadIdx.x >> 5) & 3;
+  const int row = wq * 32 + (threadIdx.x & 31);
+  const uint32_t lane_bits = (uint32_t)(wq * 32) << 16;
+  uint32_t n_pv[2] = {0u, 0u};  // PVs of each sub-tile so far
+  for (int k = 0;; ++k) {
+    const int idx = item_index(k);
+    if (idx >= p.n_items) break;
+    const WorkItem it = p.items[idx];
+    const SeqRec sr = p.seqs[it.b];
+#pragma unroll 1
+    for (int sub = 0; sub < 2; ++sub) {
+      const int64_t r0 = (int64_t)it.qblk * kBlockM + sub * kTileM;
+      const TileRange tr = tile_range(sr, r0);
+      const int i = (int)(r0 + row);
+      const bool row_valid = i < sr.sq;
+      if (!wait_warp(&ctl->epi_full[sub], k & 1u, w, kSiteEpi)) return;
+      const float inv_l = inv_l_sm[sub * kTileM + row];
+      mbar_arrive(&ctl->stat_free[sub]);
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + it.b * p.o_sb +
+                            it.h * p.o_sh + ((int64_t)sr.q_off + i) * p.o_st;
+      if (tr.hi > tr.lo) {
+        n_pv[sub] += (uint32_t)(tr.hi - tr.lo);
+        if (!wait_warp(&ctl->o_pv[sub], (n_pv[sub] - 1) & 1u, w, kSiteOPv)) return;
+        tc_fence_after();
+        const uint32_t tO = tmem + lane_bits + C::col_o(sub);
 #pragma unroll 1
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t ov[32];
           tmem_ld32_wait(tO + ch * 32u, ov);
+          uint4 pkd[4];
+          uint32_t* pw = reinterpret_cast<uint32_t*>(pkd);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
-          tmem_st32(tO + ch * 32u, ov);
+          for (int c = 0; c < 16; ++c)
+            pw[c] = pack_bf16(__uint_as_float(ov[2 * c]) * inv_l,
+                              __uint_as_float(ov[2 * c + 1]) * inv_l);
+          if (row_valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = pkd[v];
+          }
         }
-      }
-      const float ref = (m_used == -INFINITY) ? 0.f : m_used;
-      l += partial ? exp_store_p<false>(x, scale_log2, ref, tS, &ctl->p_full[sub])
-                   : exp_store_p<true>(x, scale_log2, ref, tS, &ctl->p_full[sub]);
-    }
-    if (!ok) break;
-    // Epilogue: O / l -> bf16, lse = ln(sum exp(scale q.k)).
-    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + it.b * p.o_sb +
-                          it.h * p.o_sh + ((int64_t)sr.q_off + i) * p.o_st;
-    float lse = -INFINITY;
-    if (tr.hi > tr.lo) {
-      if (!wait_warp(&ctl->o_done[sub], o_count & 1u, w, kSiteODone)) {
-        ok = false;
-        break;
-      }
-      ++o_count;
-      tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+        tc_fence_before();
+        mbar_arrive(&ctl->o_free[sub]);
+      } else if (row_valid) {
+        uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll 1
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t ov[32];
-        tmem_ld32_wait(tO + ch * 32u, ov);
-        uint4 pkd[4];
-        uint32_t* pw = reinterpret_cast<uint32_t*>(pkd);
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          pw[c] = pack_bf16(__uint_as_float(ov[2 * c]) * inv_l,
-                            __uint_as_float(ov[2 * c + 1]) * inv_l);
-        if (row_valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = pkd[v];
-        }
+        for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
       }
-      if (l > 0.f) lse = (m_used + log2f(l)) * 0.69314718055994530942f;
-    } else if (row_valid) {
-      uint4* dst = reinterpret_cast<uint4*>(orow);
-#pragma unroll 1
-      for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
     }
-    if (row_valid) p.lse[it.b * p.l_sb + it.h * p.l_sh + sr.q_off + i] = lse;
   }
 }
 
@@ -761,23 +1011,34 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100(const __grid_constan
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + C::kQBytes;
-  auto* ctl = reinterpret_cast<Ctl<C::kStages>*>(sKV + C::kKVBytes);
+  uint8_t* sP = sKV + C::kKVBytes;
+  auto* ctl = reinterpret_cast<Ctl<C::kStages>*>(sP + C::kPBytes);
+  static_assert(sizeof(Ctl<C::kStages>) <= C::kCtlBytes, "barrier area");
+  float* inv_l_sm = reinterpret_cast<float*>(sP + C::kPBytes + C::kCtlBytes);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(&ctl->q_full, 1);
-    mbar_init(&ctl->q_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&ctl->q_full[s], 1);
+      mbar_init(&ctl->q_empty[s], 1);
+    }
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&ctl->kv_full[s], 1);
       mbar_init(&ctl->kv_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ctl->s_full[s], 1);
+      mbar_init(&ctl->s_free[s], 128);
       mbar_init(&ctl->p_full[s], 128);
-      mbar_init(&ctl->o_done[s], 1);
+      mbar_init(&ctl->o_pv[s], 1);
+      mbar_init(&ctl->mufu[s], 4);  // one arrival per warp
+      mbar_init(&ctl->epi_full[s], 128);
+      mbar_init(&ctl->stat_free[s], 128);
+      mbar_init(&ctl->o_free[s], 128);
     }
     mbar_init(&ctl->drain[0], 1);
+    mbar_init(&ctl->drain[1], 1);
     ctl->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -797,12 +1058,14 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100(const __grid_constan
 
   if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-    softmax_role<D>(p, ctl, tmem, warp >> 2, w);
+    softmax_role<D>(p, ctl, inv_l_sm, tmem, sP, warp >> 2, w);
   } else if (warp < 12) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsIdle));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
+    epilogue_role<D>(p, ctl, inv_l_sm, tmem, w);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
-    if (warp == kWarpMma && lane == 0) mma_role<D>(p, ctl, tmem, sQ, sKV, w);
+    if (warp == kWarpMma && lane == 0) qk_role<D>(p, ctl, tmem, sQ, sKV, w);
+    if (warp == kWarpPv && lane == 0) pv_role<D>(p, ctl, tmem, sP, sKV, w);
     if (warp == kWarpLoad && lane == 0) load_role<D>(p, ctl, sQ, sKV, w);
   }
   __syncwarp();
