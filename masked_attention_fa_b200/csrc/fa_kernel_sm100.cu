@@ -193,6 +193,9 @@ __device__ __forceinline__ void ex2_poly_x2(float& a, float& b) {
 // without masked entries; the rest use ex2.approx on the MUFU unit.
 constexpr int kPolyPer8 = 0;
 
+// Keys of a row exponentiated before the exponential-unit turn passes on.
+constexpr int kTokenCol = 128;
+
 // Row maximum of 128 scores: eight independent chains of 3-input maxima.
 __device__ __forceinline__ float row_max128(const float (&x)[128]) {
   float m[8];
@@ -730,14 +733,11 @@ __device__ __forceinline__ void load_scores(uint32_t tS, float (&x)[128], bool p
 // x <- 2^(x * scale_log2 - ref) for the 128 keys of the row, packed into 64
 // bf16 pairs (even key in the low half); returns the row sum of the fp32
 // values (eight independent partial sums).
-template <bool kPoly>
-__device__ __forceinline__ float exp_pack(const float (&x)[128], float scale_log2, float ref,
-                                          uint32_t (&pk)[64]) {
-  const uint64_t m2 = pack_f32x2(scale_log2, scale_log2);
-  const uint64_t c2 = pack_f32x2(-ref, -ref);
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+template <bool kPoly, int kC0 = 0, int kC1 = 128>
+__device__ __forceinline__ void exp_pack_part(const float (&x)[128], uint64_t m2, uint64_t c2,
+                                              float (&acc)[8], uint32_t (&pk)[64]) {
 #pragma unroll
-  for (int c = 0; c < 128; c += 2) {
+  for (int c = kC0; c < kC1; c += 2) {
     float a = x[c], b = x[c + 1];
     fma_x2(a, b, m2, c2);
     if (kPoly && (c & 7) < kPolyPer8) {
@@ -750,6 +750,9 @@ __device__ __forceinline__ float exp_pack(const float (&x)[128], float scale_log
     add_x2(acc[2 * k], acc[2 * k + 1], a, b);
     pk[c >> 1] = pack_bf16(a, b);
   }
+}
+
+__device__ __forceinline__ float sum_acc(float (&acc)[8]) {
   add_x2(acc[0], acc[1], acc[2], acc[3]);
   add_x2(acc[4], acc[5], acc[6], acc[7]);
   add_x2(acc[0], acc[1], acc[4], acc[5]);
@@ -889,12 +892,21 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
         break;
       }
       const float ref = ((m_used == -INFINITY) ? 0.f : m_used) + zero;
+      const uint64_t m2 = pack_f32x2(scale_log2, scale_log2);
+      const uint64_t c2 = pack_f32x2(-ref, -ref);
       uint32_t pk[64];
-      const float lsum = partial ? exp_pack<false>(x, scale_log2, ref, pk)
-                                 : exp_pack<true>(x, scale_log2, ref, pk);
-      l += lsum;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // The other warpgroup gets its turn once the first kTokenCol keys are
+      // done, so both feed the exponential unit across the handover.
+      if (partial) exp_pack_part<false, 0, kTokenCol>(x, m2, c2, acc, pk);
+      else exp_pack_part<true, 0, kTokenCol>(x, m2, c2, acc, pk);
       __syncwarp();
-      if (lane == 0) arrive_token(&ctl->mufu[sub ^ 1], lsum);
+      if (lane == 0)
+        arrive_token(&ctl->mufu[sub ^ 1], ((acc[0] + acc[1]) + (acc[2] + acc[3])) +
+                                              ((acc[4] + acc[5]) + (acc[6] + acc[7])));
+      if (partial) exp_pack_part<false, kTokenCol, 128>(x, m2, c2, acc, pk);
+      else exp_pack_part<true, kTokenCol, 128>(x, m2, c2, acc, pk);
+      l += sum_acc(acc);
       if (pv_count > 0) {
         // The previous PV of this sub-tile must be done: it still reads the
         // P buffer, and O_s must hold it before it is rescaled.
