@@ -141,6 +141,31 @@ def test_visibility_probe_is_exact(case, D):
     np.testing.assert_allclose(lse_row[cnt > 0], np.log(cnt[cnt > 0]), rtol=0, atol=TOL_LSE)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("growth", ["rising", "falling"])
+def test_running_max_rescale_paths(growth, D):
+    """Keys whose norm rises (falls) along the sequence, with large logits
+    (up to ~60 at scale 1/sqrt(D)): the running maximum of a row moves up
+    tile after tile, so the lazy rescale of O is taken on many tiles (or only
+    on the first); both must match the oracle."""
+    layout, B, N, Sq, Skv = "BNSD", 1, 2, 256, 1200
+    inp = random_inputs(layout, B, N, Sq, Skv, D, seed=77)
+    j = torch.arange(Skv, dtype=torch.float32)
+    f = 1 + 5 * j / Skv if growth == "rising" else 6 - 5 * j / Skv
+    k = (inp["k"].float() * f.view(1, 1, Skv, 1)).to(torch.bfloat16)
+    q = (inp["q"].float() * 3).to(torch.bfloat16)
+    kw = _kw(layout, B, N, Sq, Skv, D, 0)  # mode 0 without a mask: every key visible
+    check_against_oracle(kw, {"q": q, "k": k, "v": inp["v"]})
+
+
+@pytest.mark.parametrize("scale", [0.05, 0.3])
+def test_explicit_scale(scale):
+    """A scale other than 1/sqrt(D) is applied to q.k before the softmax."""
+    kw = _kw("BSND", 2, 2, 300, 420, 128, 3, scale=scale)
+    inp = random_inputs("BSND", 2, 2, 300, 420, 128, seed=91)
+    check_against_oracle(kw, inp)
+
+
 def test_deterministic_bitwise():
     kw = _kw("BNSD", 2, 4, 700, 900, 128, 3)
     inp = random_inputs("BNSD", 2, 4, 700, 900, 128, seed=11)
