@@ -72,6 +72,10 @@ def _load():
         lib.oracle_attn_rows.restype = ctypes.c_int
         lib.oracle_mask.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, i64, i64, P]
         lib.oracle_mask.restype = None
+        lib.oracle_tile_classes.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, i64, i64, i64, P]
+        lib.oracle_tile_classes.restype = None
+        lib.oracle_tile_ranges.argtypes = [P, i64, i64, P]
+        lib.oracle_tile_ranges.restype = None
         lib.oracle_visible_count.argtypes = [ctypes.POINTER(_Desc), P, P, P, P]
         lib.oracle_visible_count.restype = ctypes.c_int64
         lib.oracle_flash_tiled.argtypes = [P, P, P, P, i64, i64, i64, i64, ctypes.c_double, P]
@@ -171,6 +175,31 @@ def mask_matrix(pb: Problem, b: int, h: int = 0) -> np.ndarray:
     pre, cq, ckv, m = pb._ptrs()
     if sq > 0 and skv > 0:
         _load().oracle_mask(ctypes.byref(d), pre, cq, ckv, m, b, h, out.ctypes.data)
+    return out
+
+
+def tile_classes(pb: Problem, b: int, h: int = 0, tile: int = 128) -> np.ndarray:
+    """Block occupancy of sequence b, head h: [ceil(Sq_b/tile), ceil(Skv_b/tile)]
+    uint8, 0 = no visible pair, 2 = every existing row sees every key of the
+    block (all keys existing), 1 = otherwise."""
+    _, _, sq, skv = pb.seq(b)
+    out = np.zeros(((max(sq, 0) + tile - 1) // tile, (max(skv, 0) + tile - 1) // tile),
+                   dtype=np.uint8)
+    d = pb.desc()
+    pre, cq, ckv, m = pb._ptrs()
+    if out.size:
+        _load().oracle_tile_classes(ctypes.byref(d), pre, cq, ckv, m, b, h, tile,
+                                    out.ctypes.data)
+    return out
+
+
+def tile_ranges(classes) -> np.ndarray:
+    """Per query block of a class matrix: (lo, hi, full_lo, full_hi) int32."""
+    c = np.ascontiguousarray(np.asarray(classes, dtype=np.uint8))
+    n_qt, n_kt = c.shape
+    out = np.zeros((n_qt, 4), dtype=np.int32)
+    if n_qt:
+        _load().oracle_tile_ranges(c.ctypes.data, n_qt, n_kt, out.ctypes.data)
     return out
 
 

@@ -16,6 +16,11 @@
  *   - The attention itself as its plain definition: S = scale * Q K^T,
  *     softmax over the visible keys of each row, O = P V, and the per-row
  *     natural log-sum-exp. A row with no visible key gives O = 0, lse = -inf.
+ *   - The occupancy of the visibility matrix by 128 x 128 blocks (which
+ *     blocks hold no visible pair, which hold only visible pairs) and the
+ *     range of key blocks each query block must visit: the sparseMode page
+ *     has the operator compute only the part the mask and the band leave
+ *     visible, and these are that statement summarised by block.
  *   - The tiled online-softmax recurrence (running max m_i, running sum l_i,
  *     normalised output) of the "FlashAttention tiling & online softmax"
  *     exercise page (section "Mục tiêu kiến thức"), used only to pin the
@@ -326,6 +331,81 @@ void oracle_mask(const oracle_desc* d, const int64_t* prefix,
         for (int64_t j = 0; j < s.skv; ++j)
             out[i * s.skv + j] = (uint8_t)oracle_visible(d, prefix, cu_q,
                                                          cu_kv, mask, b, h, i, j);
+}
+
+/*
+ * Occupancy of the visibility matrix of sequence b, head h, summarised by
+ * blocks of `tile` query rows x `tile` keys: out[qt * n_kt + kt] with
+ * n_kt = ceil(Skv_b / tile) is
+ *   0  when no pair of the block is visible,
+ *   2  when every row of the block that exists (i < Sq_b) sees every one of
+ *      the block's `tile` keys and all of them exist (j < Skv_b),
+ *   1  otherwise.
+ * This is what an attention over the matrix may skip (0) or compute without
+ * looking at the mask (2); it follows from the visibility rule alone.
+ */
+void oracle_tile_classes(const oracle_desc* d, const int64_t* prefix,
+                         const int64_t* cu_q, const int64_t* cu_kv,
+                         const uint8_t* mask, int64_t b, int64_t h,
+                         int64_t tile, uint8_t* out) {
+    seq_info s = seq_of(d, cu_q, cu_kv, b);
+    const int64_t n_qt = (s.sq + tile - 1) / tile;
+    const int64_t n_kt = (s.skv + tile - 1) / tile;
+    for (int64_t qt = 0; qt < n_qt; ++qt) {
+        for (int64_t kt = 0; kt < n_kt; ++kt) {
+            int any = 0, all = 1;
+            for (int64_t i = qt * tile; i < (qt + 1) * tile && i < s.sq; ++i) {
+                for (int64_t j = kt * tile; j < (kt + 1) * tile; ++j) {
+                    const int v = j < s.skv &&
+                                  oracle_visible(d, prefix, cu_q, cu_kv, mask,
+                                                 b, h, i, j);
+                    any |= v;
+                    all &= v;
+                }
+            }
+            out[qt * n_kt + kt] = (uint8_t)(any ? (all ? 2 : 1) : 0);
+        }
+    }
+}
+
+/*
+ * The key-block range each query block of a class matrix (as written by
+ * oracle_tile_classes, n_qt x n_kt) has to visit: out[4 qt + 0..3] =
+ *   lo, hi         the first non-empty block and one past the last one;
+ *   full_lo, full_hi  the longest run of consecutive class-2 blocks, the
+ *                  earliest of equally long runs, or lo, lo when there is
+ *                  no class-2 block.
+ * A query block whose blocks are all empty gets 0, 0, 0, 0.
+ */
+void oracle_tile_ranges(const uint8_t* cls, int64_t n_qt, int64_t n_kt,
+                        int32_t* out) {
+    for (int64_t qt = 0; qt < n_qt; ++qt) {
+        const uint8_t* c = cls + qt * n_kt;
+        int64_t lo = -1, hi = 0, best_lo = 0, best_len = 0;
+        for (int64_t kt = 0; kt < n_kt; ++kt) {
+            if (c[kt] != 0) {
+                if (lo < 0) lo = kt;
+                hi = kt + 1;
+            }
+            if (c[kt] == 2 && (kt == 0 || c[kt - 1] != 2)) {
+                int64_t e = kt;
+                while (e < n_kt && c[e] == 2) ++e;
+                if (e - kt > best_len) {
+                    best_len = e - kt;
+                    best_lo = kt;
+                }
+            }
+        }
+        int32_t* r = out + 4 * qt;
+        if (lo < 0) {
+            r[0] = r[1] = r[2] = r[3] = 0;
+        } else {
+            r[0] = (int32_t)lo;
+            r[1] = (int32_t)hi;
+            r[2] = (int32_t)(best_len > 0 ? best_lo : lo);
+            r[3] = (int32_t)(best_len > 0 ? best_lo + best_len : lo);
+        }
+    }
 }
 
 /* Number of visible (b, h, i, j) pairs, by enumeration. */

@@ -449,3 +449,111 @@ def test_tiled_recurrence_with_masks_matches_masked_softmax():
         for blk in (1, 2, 3, 5, 11):
             out = oracle.flash_tiled(q, k, v, block_size=blk, vis=vis)
             np.testing.assert_allclose(out, o[:, 0], rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Block occupancy of the visibility matrix (what the attention may skip or
+# compute without the element mask) and the key-block range per query block.
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("nb", [1, 4])
+def test_tile_classes_of_causal_are_the_triangle(nb):
+    """leftUpCausal on a square of nb x nb whole blocks: blocks below the
+    diagonal are all visible, diagonal blocks mixed, blocks above it empty."""
+    S = 128 * nb
+    pb = Problem("BNSD", 1, 1, S, S, 8, sparse_mode=2)
+    qt, kt = np.meshgrid(np.arange(nb), np.arange(nb), indexing="ij")
+    want = np.where(kt < qt, 2, np.where(kt == qt, 1, 0)).astype(np.uint8)
+    assert np.array_equal(oracle.tile_classes(pb, 0), want)
+    r = oracle.tile_ranges(want)
+    for q in range(nb):
+        assert r[q].tolist() == [0, q + 1, 0, q]
+
+
+@pytest.mark.parametrize("pre", [300, 10 ** 6])
+def test_tile_classes_of_band_mask_zero_equal_causal(pre):
+    """sparseMode 0 with an all-zero mask, nextTokens 0 and preTokens >= Sq is
+    causal (the page's "causal via band"), block by block."""
+    S = 256
+    zero = np.zeros((S, S), dtype=np.uint8)
+    pb0 = Problem("BNSD", 1, 1, S, S, 8, sparse_mode=0, pre_tokens=pre, next_tokens=0,
+                  mask=zero, mask_kind="SS")
+    pb2 = Problem("BNSD", 1, 1, S, S, 8, sparse_mode=2)
+    assert np.array_equal(oracle.tile_classes(pb0, 0), oracle.tile_classes(pb2, 0))
+
+
+def test_tile_classes_of_open_and_closed_masks():
+    """allMask with nothing masked: whole key blocks are full, the ragged last
+    key block (keys past Skv) is mixed; everything masked: all empty."""
+    Sq, Skv = 300, 333
+    open_ = Problem("BNSD", 1, 1, Sq, Skv, 8, sparse_mode=1,
+                    mask=np.zeros((Sq, Skv), np.uint8), mask_kind="SS")
+    want = np.array([[2, 2, 1]] * 3, dtype=np.uint8)
+    assert np.array_equal(oracle.tile_classes(open_, 0), want)
+    assert oracle.tile_ranges(want).tolist() == [[0, 3, 0, 2]] * 3
+    shut = Problem("BNSD", 1, 1, Sq, Skv, 8, sparse_mode=1,
+                   mask=np.ones((Sq, Skv), np.uint8), mask_kind="SS")
+    assert not oracle.tile_classes(shut, 0).any()
+    assert not oracle.tile_ranges(np.zeros((3, 3), np.uint8)).any()
+
+
+def test_tile_classes_of_a_constructed_block_mask():
+    """Blocks of 4 on a 10 x 13 allMask, each block set up to have a known
+    class: whole-visible (2), one visible pair (1), one hidden pair (1),
+    visible rows that end at Sq (2: rows past Sq do not exist), visible keys
+    that end at Skv (1: the block's keys past Skv do not exist), hidden (0).
+    Per batch and head (BNSS) the classes follow that plane's mask."""
+    Sq, Skv, t = 10, 13, 4
+    m = np.ones((2, 1, Sq, Skv), dtype=np.uint8)
+    m[0, 0, 0:4, 0:4] = 0          # (0, 0) full
+    m[0, 0, 1, 6] = 0              # (0, 1) one visible pair
+    m[0, 0, 4:8, 8:12] = 0         # (1, 2) full ...
+    m[0, 0, 5, 9] = 1              # ... but one hidden pair: mixed
+    m[0, 0, 8:10, 0:4] = 0         # (2, 0) rows 8, 9 only: full
+    m[0, 0, 8:10, 12] = 0          # (2, 3) key 12 only: mixed
+    m[1, 0, 4:8, 4:8] = 0          # batch 1: (1, 1) full
+    pb = Problem("BNSD", 2, 1, Sq, Skv, 8, sparse_mode=1, mask=m, mask_kind="B1SS")
+    want0 = np.zeros((3, 4), np.uint8)
+    want0[0, 0], want0[0, 1], want0[1, 2], want0[2, 0], want0[2, 3] = 2, 1, 1, 2, 1
+    assert np.array_equal(oracle.tile_classes(pb, 0, tile=t), want0)
+    want1 = np.zeros((3, 4), np.uint8)
+    want1[1, 1] = 2
+    assert np.array_equal(oracle.tile_classes(pb, 1, tile=t), want1)
+    assert oracle.tile_ranges(want0).tolist() == [[0, 2, 0, 1], [2, 3, 2, 2], [0, 4, 0, 1]]
+    assert oracle.tile_ranges(want1).tolist() == [[0, 0, 0, 0], [1, 2, 1, 2], [0, 0, 0, 0]]
+
+
+@pytest.mark.parametrize("row,want", [
+    ([0, 1, 2, 2, 0, 2, 2, 2, 1, 0], [1, 9, 5, 8]),   # longest full run wins
+    ([2, 2, 0, 2, 2], [0, 5, 0, 2]),                  # equal runs: the first
+    ([1, 0, 1], [0, 3, 0, 0]),                        # no full block: lo, lo
+    ([0, 0, 2], [2, 3, 2, 3]),
+    ([0, 0, 0], [0, 0, 0, 0]),                        # nothing visible
+])
+def test_tile_ranges_hand_cases(row, want):
+    assert oracle.tile_ranges(np.array([row], np.uint8)).tolist() == [want]
+
+
+def test_tile_classes_match_bruteforce_blocks():
+    """Against the visibility matrix cut into blocks by numpy, over every
+    sparseMode on a small ragged shape with tile 5."""
+    rng = np.random.default_rng(3)
+    Sq, Skv, t = 17, 23, 5
+    for mode, extra in [(0, dict(pre_tokens=6, next_tokens=2)), (1, {}), (2, {}), (3, {}),
+                        (4, dict(pre_tokens=7, next_tokens=1))]:
+        mask = None
+        if mode <= 1:
+            mask = (rng.random((Sq, Skv)) < 0.2).astype(np.uint8)
+            mask[:, 15:] = 0                       # some whole-visible blocks
+            mask[10:15, :] = 1                     # a hidden block row
+        pb = Problem("BNSD", 1, 1, Sq, Skv, 8, sparse_mode=mode, mask=mask,
+                     mask_kind="SS" if mask is not None else None, **extra)
+        vis = oracle.mask_matrix(pb, 0).astype(bool)
+        pad = np.zeros((-(-Sq // t) * t, -(-Skv // t) * t), dtype=bool)
+        pad[:Sq, :Skv] = vis
+        got = oracle.tile_classes(pb, 0, tile=t)
+        for qt in range(got.shape[0]):
+            for kt in range(got.shape[1]):
+                blk = pad[qt * t:min((qt + 1) * t, Sq), kt * t:(kt + 1) * t]
+                cls = 2 if blk.all() else (1 if blk.any() else 0)
+                assert got[qt, kt] == cls, (mode, qt, kt)
