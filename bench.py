@@ -155,16 +155,36 @@ def visible_pairs(w, has_mask, mask_host=None):
     if has_mask:
         import numpy as np
         import torch
-        m = mask_host.to(torch.bool).numpy()
-        S = w.Sq
-        ii = np.arange(S)[:, None]
-        jj = np.arange(w.Skv)[None, :]
-        band = (ii - jj <= w.pre_tokens) & (jj - ii <= w.next_tokens)
-        per = int(((~m) & band).sum()) if m.ndim == 2 else int(((~m) & band).sum())
-        return per * (w.N * w.B if m.ndim == 2 else 1)
+        vis = ~mask_host.to(torch.bool).numpy()
+        if w.sparse_mode == 0:  # mode 0: the mask inside the preTokens/nextTokens band
+            ii = np.arange(w.Sq)[:, None]
+            jj = np.arange(w.Skv)[None, :]
+            vis = vis & ((ii - jj <= w.pre_tokens) & (jj - ii <= w.next_tokens))
+        # planes: SS one for every (b, h), B1SS one per b, BNSS one per (b, h)
+        mult = {"SS": w.B * w.N, "B1SS": w.N, "BNSS": 1}[w.mask_kind]
+        return int(vis.sum()) * mult
     d = fa.make_desc(w.layout, w.B, w.N, w.Sq, w.Skv, w.D, w.sparse_mode, w.pre_tokens,
                      w.next_tokens, w.scale, w.mask_kind)
     return fa.fa_visible_pairs(d, **workload_args(w))
+
+
+def prepass_bytes(w):
+    """Algorithmic bytes of the dense-mask pre-pass: every mask byte of the
+    128 x 128 tiles inside the band (the geometry's non-EMPTY tiles, cut at
+    Sq and Skv) is read once, per mask plane; plus one class byte per tile
+    written and read again, and 16 bytes of range per 128-row query block."""
+    import masked_attention_fa_b200 as fa
+    d = fa.make_desc(w.layout, w.B, w.N, w.Sq, w.Skv, w.D, w.sparse_mode, w.pre_tokens,
+                     w.next_tokens, w.scale, w.mask_kind)
+    planes = {"SS": 1, "B1SS": w.B, "BNSS": w.B * w.N}[w.mask_kind]
+    n_qt, n_kt = (w.Sq + 127) // 128, (w.Skv + 127) // 128
+    per_plane = 0
+    for qt in range(n_qt):
+        rows = min(128, w.Sq - 128 * qt)
+        for kt in range(n_kt):
+            if fa.fa_tile_class(d, 0, qt, kt, has_mask=True) != fa.FA_TILE_EMPTY:
+                per_plane += rows * min(128, w.Skv - 128 * kt)
+    return planes * (per_plane + 2 * n_qt * n_kt + 16 * n_qt)
 
 
 def cpu_baseline_sample(w, inputs, seconds):
@@ -282,8 +302,28 @@ def main():
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
+    # Dense-mask workloads: the step is the library's occupancy pre-pass
+    # followed by the attention on its ranges (the same two stages fa_fwd
+    # runs internally), with an event between them so each kernel is timed.
+    dense = mask is not None
+    if dense:
+        cls_shape, rng_shape = fa.occupancy_shapes(attn.desc)
+        tile_cls = torch.empty(cls_shape, dtype=torch.uint8, device=dev)
+        ranges = torch.empty(rng_shape, dtype=torch.int32, device=dev)
+
+    def prepass():
+        fa.fa_mask_occupancy(attn.desc, mask, tile_class=tile_cls, ranges=ranges, stream=stream)
+
+    def attention():
+        if dense:
+            attn(q, k, v, atten_mask=mask, out=o, lse=lse, stream=stream, ranges=ranges)
+        else:
+            attn(q, k, v, atten_mask=mask, out=o, lse=lse, stream=stream, **arrays)
+
     def step():
-        attn(q, k, v, atten_mask=mask, out=o, lse=lse, stream=stream, **arrays)
+        if dense:
+            prepass()
+        attention()
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -297,11 +337,15 @@ def main():
         dist.barrier()
     torch.cuda.synchronize(dev)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     for i in range(args.steps):
         flush.fill_(float(i))
         starts[i].record(stream)
-        step()
+        if dense:
+            prepass()
+        mids[i].record(stream)
+        attention()
         ends[i].record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
@@ -310,6 +354,9 @@ def main():
     attn.sync_status()
     times_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms = sum(times_ms) / len(times_ms)
+    # the attention kernel alone (the whole step when there is no pre-pass)
+    kern_ms = sum(m.elapsed_time(e) for m, e in zip(mids, ends)) / len(mids)
+    pre_ms = sum(s.elapsed_time(m) for s, m in zip(starts, mids)) / len(mids)
     t = torch.tensor([ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -356,12 +403,25 @@ def main():
     if rank == 0:
         peaks, peak_src = load_peaks()
         peak = float(peaks["bf16_tflops"])
-        achieved = flops / (ms * 1e-3) / 1e12
+        achieved = flops / (kern_ms * 1e-3) / 1e12
         traffic = load_traffic(w.name)
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": traffic,
                     "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
-                    "kernel": f"fa_fwd_sm100<{w.D}>"}
+                    "kernel": f"fa_fwd_sm100<{w.D}, {'true' if dense else 'false'}>",
+                    "kernel_ms": kern_ms}
+        if dense:
+            roofline["kernel_ms_includes"] = ("the one-block work-list rebuild "
+                                              "(occupancy_schedule) launched just before it")
+        prepass_line = None
+        if dense:
+            mbytes = prepass_bytes(w)
+            gbs = mbytes / (pre_ms * 1e-3) / 1e9
+            hbm = float(peaks["hbm_gbs"])
+            prepass_line = {"kernels": "occupancy_strips", "ms": pre_ms,
+                            "bound": "hbm", "bytes": mbytes, "achieved": gbs, "peak": hbm,
+                            "unit": "GB/s", "frac": gbs / hbm,
+                            "peak_source": f"{peak_src} hbm_gbs"}
         cpu = None
         if not args.no_cpu_baseline and world == 1:
             tf, cores, desc = cpu_baseline_sample(w, inputs, args.cpu_seconds)
@@ -378,8 +438,10 @@ def main():
                            "parallelism": f"replicas x{world}"},
                 "frac_of_peak": value / world / peak,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": args.steps, "clocks": clocks,
+                "gpu_launches": args.steps * (4 if dense else 1), "clocks": clocks,
                 "ms_min": min(times_ms), "ms_median": statistics.median(times_ms)}
+        if prepass_line is not None:
+            line["prepass"] = prepass_line
         print(json.dumps(line))
     attn.close()
     if world > 1:

@@ -126,6 +126,14 @@ fa_status_t fa_create(const fa_desc_t* desc, fa_handle_t* out);
  * sequence with Sq_b > 0: pre >= Skv_b and next >= Sq_b - Skv_b. Violations
  * return FA_ERR_PARAM_INVALID before any device work.
  *
+ * Dense masks (mode 1, or mode 0 with atten_mask): the call first runs the
+ * occupancy pre-pass of fa_mask_occupancy into the handle's workspace (two
+ * small kernels on the same stream), so that key tiles the mask hides
+ * entirely are skipped and tiles it leaves entirely visible are computed
+ * without reading it, then a one-block kernel that rebuilds the work list
+ * from the pre-pass's ranges, longest item first by its real number of key
+ * tiles; fa_fwd_with_ranges skips the pre-pass but not the rebuild.
+ *
  * Asynchronous: returns once the kernel is enqueued. The host arrays are
  * read during the call only. Device-side problems (a wait that gave up) are
  * reported by fa_sync_status. The device must be sm_100 (B200 class);
@@ -167,6 +175,12 @@ int32_t fa_version(void);
  * Capacity: 256 + 32 * B (rounded up to 256) + 16 * items bytes, where items
  * = N * sum over sequences of ceil(Sq_b / 256); a problem beyond 1 MiB returns
  * FA_ERR_UNSUPPORTED before any device work (use fa_create/fa_fwd then).
+ * A dense-mask call puts each item's two key-tile ranges (32 bytes per item,
+ * rounded up to 256) and the occupancy pre-pass's scratch (16 bytes per mask
+ * plane and 128-row query block, rounded up to 256, plus 1 byte per plane
+ * and 128 x 128 tile) behind the work list when they fit; when they do not,
+ * the call runs without the pre-pass (every tile of the band with the
+ * element mask) and gives the same result.
  * Sharing: every call shares the array and leaves its work list there; the
  * error word is cleared at the start of each call. Calls whose kernels
  * overlap on the GPU race on the array: order them on one stream. Host calls
@@ -181,6 +195,60 @@ fa_status_t fa_fwd_noalloc(const fa_desc_t* desc, const void* q, const void* k, 
                            const uint8_t* atten_mask, const int64_t* prefix,
                            const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
                            void* o, float* lse, void* cuda_stream);
+
+/*
+ * fa_mask_occupancy — the dense-mask pre-pass that fa_fwd and
+ * fa_fwd_noalloc run before the attention kernel in sparseMode 1 (allMask)
+ * and in sparseMode 0 with an attenMask ("sparseMode参数说明" page,
+ * sparseMode=0 and sparseMode=1 sections: the operator computes the pairs
+ * the mask leaves visible, in mode 0 only those inside the preTokens /
+ * nextTokens band), enqueued on its own on `cuda_stream`.
+ *
+ * The mask has P planes of Sq x Skv bytes (SS: P = 1, B1SS: P = B, BNSS:
+ * P = B * N; nonzero = masked). For plane p, query rows [128 qt, 128 qt + 128)
+ * and keys [128 kt, 128 kt + 128), a pair (i, j) is visible when i < Sq,
+ * j < Skv, the mode's band admits it and the mask byte is 0. Outputs:
+ * tile_class  device uint8 [P, ceil(Sq/128), ceil(Skv/128)]:
+ *             FA_TILE_EMPTY (no visible pair), FA_TILE_FULL (every row
+ *             i < Sq of the tile sees all 128 keys, each < Skv) or
+ *             FA_TILE_PARTIAL.
+ * ranges      device int32 [P, ceil(Sq/128), 4], 16-byte aligned: per query
+ *             sub-tile {lo, hi, full_lo, full_hi}: [lo, hi) runs from the
+ *             first to the last non-EMPTY tile ({0, 0, 0, 0} when all are
+ *             EMPTY) and [full_lo, full_hi) is the longest run of FULL tiles,
+ *             the first one on ties (full_lo = full_hi = lo when there is
+ *             none). fa_fwd visits the tiles of [lo, hi) and applies the
+ *             element mask outside [full_lo, full_hi).
+ * desc        layout BNSD or BSND, sparse_mode 0 or 1 with a mask_kind;
+ *             the other checks are fa_create's. atten_mask: device, in the
+ *             mask_kind shape. All buffers belong to the caller.
+ * Errors: FA_ERR_NULLPTR, FA_ERR_PARAM_INVALID (other modes, no mask kind,
+ * unaligned ranges), FA_ERR_UNSUPPORTED (not sm_100, TND), FA_ERR_CUDA
+ * (launch). Asynchronous like fa_fwd; it reads the whole mask inside the
+ * band once (1 byte per element).
+ */
+fa_status_t fa_mask_occupancy(const fa_desc_t* desc, const uint8_t* atten_mask,
+                              uint8_t* tile_class, int32_t* ranges, void* cuda_stream);
+
+/*
+ * fa_fwd_with_ranges — fa_fwd for a dense-mask handle (sparse_mode 1, or 0
+ * with a mask_kind) that takes the pre-pass's ranges from the caller instead
+ * of running the pre-pass: one fa_mask_occupancy can then serve every call
+ * that uses the same mask (for example every layer of a model); the call
+ * launches the one-block work-list rebuild and the attention kernel.
+ *
+ * ranges  device int32, 16-byte aligned, exactly as fa_mask_occupancy wrote
+ *         them for this descriptor's shape and this atten_mask, which must
+ *         not have changed since; other values give undefined O and lse
+ *         (every memory access stays inside the operands all the same).
+ * The other arguments are fa_fwd's (no prefix or length arrays: modes 0/1
+ * take none). Errors as fa_fwd, plus FA_ERR_PARAM_INVALID for a handle
+ * without a dense mask or unaligned ranges and FA_ERR_NULLPTR for NULL
+ * ranges or atten_mask.
+ */
+fa_status_t fa_fwd_with_ranges(fa_handle_t h, const void* q, const void* k, const void* v,
+                               const uint8_t* atten_mask, const int32_t* ranges, void* o,
+                               float* lse, void* cuda_stream);
 
 /* ---------------- host-only helpers (no device work) ------------------- */
 

@@ -101,6 +101,10 @@ def load_library():
     lib.fa_plan_stats.restype = st
     lib.fa_fwd_noalloc.argtypes = [dp, P, P, P, P, i64p, i64p, i64p, P, P, P]
     lib.fa_fwd_noalloc.restype = st
+    lib.fa_mask_occupancy.argtypes = [dp, P, P, P, P]
+    lib.fa_mask_occupancy.restype = st
+    lib.fa_fwd_with_ranges.argtypes = [P, P, P, P, P, P, P, P, P]
+    lib.fa_fwd_with_ranges.restype = st
     lib.fa_split_queries.argtypes = [dp, i64p, i64p, ctypes.c_int32, i64p, ctypes.c_int32,
                                      ctypes.POINTER(fa_split_part_t), i64p, i64p]
     lib.fa_split_queries.restype = st
@@ -110,7 +114,7 @@ def load_library():
 
 EXPORTED = ("fa_create", "fa_fwd", "fa_sync_status", "fa_destroy", "fa_last_error",
             "fa_version", "fa_validate", "fa_visible_pairs", "fa_tile_class", "fa_plan_stats",
-            "fa_fwd_noalloc", "fa_split_queries")
+            "fa_fwd_noalloc", "fa_split_queries", "fa_mask_occupancy", "fa_fwd_with_ranges")
 
 
 def _check(status):
@@ -220,6 +224,47 @@ def fa_fwd(h, q, k, v, o, lse, atten_mask=None, prefix=None, actual_seq_qlen=Non
                                  _ptr(o), _ptr(lse), ctypes.c_void_p(int(stream))))
 
 
+def _stream_int(stream, device):
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
+    if hasattr(stream, "cuda_stream"):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def occupancy_shapes(desc):
+    """Shapes of fa_mask_occupancy's outputs: (tile classes, ranges)."""
+    planes = {1: 1, 2: int(desc.B), 3: int(desc.B) * int(desc.N)}[int(desc.mask_kind)]
+    n_qt = (int(desc.Sq) + 127) // 128
+    n_kt = (int(desc.Skv) + 127) // 128
+    return (planes, n_qt, n_kt), (planes, n_qt, 4)
+
+
+def fa_mask_occupancy(desc, atten_mask, tile_class=None, ranges=None, stream=None):
+    """The dense-mask pre-pass alone (see include/fa.h): returns the uint8
+    tile classes [P, ceil(Sq/128), ceil(Skv/128)] and the int32 ranges
+    [P, ceil(Sq/128), 4] as CUDA tensors (allocated unless given)."""
+    import torch
+    cshape, rshape = occupancy_shapes(desc)
+    dev = atten_mask.device
+    if tile_class is None:
+        tile_class = torch.empty(cshape, dtype=torch.uint8, device=dev)
+    if ranges is None:
+        ranges = torch.empty(rshape, dtype=torch.int32, device=dev)
+    _check(load_library().fa_mask_occupancy(ctypes.byref(desc), _ptr(atten_mask),
+                                            _ptr(tile_class), _ptr(ranges),
+                                            ctypes.c_void_p(_stream_int(stream, dev))))
+    return tile_class, ranges
+
+
+def fa_fwd_with_ranges(h, q, k, v, o, lse, atten_mask, ranges, stream=None):
+    """fa_fwd for a dense-mask handle with the pre-pass's ranges supplied."""
+    _check(load_library().fa_fwd_with_ranges(h, _ptr(q), _ptr(k), _ptr(v), _ptr(atten_mask),
+                                             _ptr(ranges), _ptr(o), _ptr(lse),
+                                             ctypes.c_void_p(_stream_int(stream, q.device))))
+
+
 def fa_fwd_noalloc(desc, q, k, v, o, lse, atten_mask=None, prefix=None, actual_seq_qlen=None,
                    actual_seq_kvlen=None, stream=None):
     """The allocation-free forward: no handle, the work list lives in the
@@ -279,7 +324,7 @@ class MaskedAttention:
         return (d.Sq, d.N, d.D), (d.N, d.Sq)
 
     def __call__(self, q, k, v, atten_mask=None, prefix=None, actual_seq_qlen=None,
-                 actual_seq_kvlen=None, out=None, lse=None, stream=None):
+                 actual_seq_kvlen=None, out=None, lse=None, stream=None, ranges=None):
         import torch
         oshape, lshape = self.out_shapes()
         if out is None:
@@ -294,9 +339,17 @@ class MaskedAttention:
         if atten_mask is not None:
             if atten_mask.dtype not in (torch.uint8, torch.bool) or not atten_mask.is_contiguous():
                 raise ValueError("atten_mask must be a contiguous uint8/bool tensor")
-        fa_fwd(self.handle, q, k, v, out, lse, atten_mask, prefix, actual_seq_qlen,
-               actual_seq_kvlen, stream)
+        if ranges is not None:
+            fa_fwd_with_ranges(self.handle, q, k, v, out, lse, atten_mask, ranges, stream)
+        else:
+            fa_fwd(self.handle, q, k, v, out, lse, atten_mask, prefix, actual_seq_qlen,
+                   actual_seq_kvlen, stream)
         return out, lse
+
+    def occupancy(self, atten_mask, stream=None):
+        """Run the dense-mask pre-pass on its own: (tile classes, ranges);
+        pass the ranges back as ``attn(..., ranges=ranges)`` to skip it."""
+        return fa_mask_occupancy(self.desc, atten_mask, stream=stream)
 
     def sync_status(self):
         st = fa_sync_status(self.handle)

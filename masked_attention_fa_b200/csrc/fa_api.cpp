@@ -28,7 +28,9 @@ struct fa_handle_s {
   bool plan_valid = false;
   int32_t n_items = 0;
   int32_t n_seqs = 0;
+  SeqRec geo0{};  // geometry of sequence 0 (every sequence's, outside TND)
   // device workspace: [error word | pad to 256 B][SeqRec x B][WorkItem x n]
+  // then, for a dense attenMask, the occupancy pre-pass's ranges and classes
   void* d_ws = nullptr;
   size_t ws_bytes = 0;
   // pinned staging of the work list and the event of its last upload
@@ -58,6 +60,35 @@ fa_status_t cuda_fail(cudaError_t e, const char* what) {
 }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Planes of the attenMask the occupancy pre-pass reduces: SS one plane for
+// every batch and head, B1SS one per batch, BNSS one per batch and head; 0
+// when the call reads no mask.
+int64_t mask_planes(const fa_desc_t* d, int has_mask) {
+  if (!has_mask) return 0;
+  if (d->mask_kind == FA_MASK_SS) return 1;
+  if (d->mask_kind == FA_MASK_B1SS) return d->B;
+  return d->B * d->N;
+}
+
+// Dense-mask calls keep, after the work list, each item's two ranges
+// (item_tr, 32 bytes per item) and then the pre-pass's scratch.
+size_t item_tr_offset(int32_t n_seqs, int32_t n_items) {
+  return align_up(kHeaderBytes + align_up((size_t)n_seqs * sizeof(SeqRec), 256) +
+                      (size_t)n_items * sizeof(WorkItem),
+                  256);
+}
+size_t occupancy_offset(int32_t n_seqs, int32_t n_items) {
+  return item_tr_offset(n_seqs, n_items) +
+         align_up((size_t)n_items * 2 * sizeof(TileRange), 256);
+}
+
+// Point the pre-pass at `scratch`: the ranges, then (256-byte aligned) the
+// classes; `a` already has its shape.
+void occupancy_bind(OccParams* a, uint8_t* scratch) {
+  a->ranges = reinterpret_cast<TileRange*>(scratch);
+  a->cls = scratch + align_up((size_t)(a->n_planes * a->n_qt) * sizeof(TileRange), 256);
+}
 
 fa_status_t bind_device(fa_handle_t h) {
   int dev = 0;
@@ -147,7 +178,12 @@ fa_status_t refresh_plan(fa_handle_t h, const int64_t* prefix, const int64_t* cu
   const size_t seq_bytes = recs.size() * sizeof(SeqRec);
   const size_t item_bytes = items.size() * sizeof(WorkItem);
   const size_t payload = align_up(seq_bytes, 256) + item_bytes;
-  fa_status_t st = ensure_workspace(h, kHeaderBytes + payload);
+  const int64_t planes = mask_planes(&h->desc, has_mask);
+  const size_t occ = planes ? occupancy_bytes(planes, h->desc.Sq, h->desc.Skv) : 0;
+  // Dense masks: item_tr and the pre-pass's scratch follow the list.
+  fa_status_t st = ensure_workspace(
+      h, planes ? occupancy_offset((int32_t)recs.size(), (int32_t)items.size()) + occ
+                : kHeaderBytes + payload);
   if (st != FA_OK) return st;
   st = ensure_stage(h, payload);
   if (st != FA_OK) return st;
@@ -169,6 +205,7 @@ fa_status_t refresh_plan(fa_handle_t h, const int64_t* prefix, const int64_t* cu
   h->plan_valid = true;
   h->n_items = (int32_t)items.size();
   h->n_seqs = (int32_t)recs.size();
+  if (!recs.empty()) h->geo0 = recs[0];
   return FA_OK;
 }
 
@@ -238,11 +275,16 @@ fa_status_t fa_create(const fa_desc_t* desc, fa_handle_t* out) {
   return FA_OK;
 }
 
-fa_status_t fa_fwd(fa_handle_t h, const void* q, const void* k, const void* v,
-                   const uint8_t* atten_mask, const int64_t* prefix,
-                   const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen, void* o,
-                   float* lse, void* cuda_stream) {
-  clear_error();
+}  // extern "C"
+
+namespace {
+
+// fa_fwd and fa_fwd_with_ranges. `ranges` (or null): the dense-mask
+// occupancy of this mask, already computed by fa_mask_occupancy.
+fa_status_t forward(fa_handle_t h, const void* q, const void* k, const void* v,
+                    const uint8_t* atten_mask, const int32_t* ranges, const int64_t* prefix,
+                    const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen, void* o,
+                    float* lse, void* cuda_stream) {
   if (!h) return fail(FA_ERR_NULLPTR, "handle is NULL");
   if (!q || !k || !v || !o || !lse) return fail(FA_ERR_NULLPTR, "q, k, v, o and lse are required");
   const fa_desc_t* d = &h->desc;
@@ -289,6 +331,47 @@ fa_status_t fa_fwd(fa_handle_t h, const void* q, const void* k, const void* v,
     p.m_sb = (d->mask_kind == FA_MASK_SS) ? 0 : (d->mask_kind == FA_MASK_B1SS ? plane : d->N * plane);
     p.m_sh = (d->mask_kind == FA_MASK_BNSS) ? plane : 0;
   }
+  if (has_mask) {
+    // Reduce the mask to per-sub-tile key-tile ranges (unless the caller
+    // already did), then rebuild the work list from them on the device, all
+    // on the same stream ahead of the attention kernel.
+    OccParams a;
+    std::memset(&a, 0, sizeof(a));
+    occupancy_shape(&a, h->geo0, mask_planes(d, has_mask));
+    a.mask = atten_mask;
+    SchedParams sp;
+    std::memset(&sp, 0, sizeof(sp));
+    sp.B = (int32_t)d->B;
+    sp.N = (int32_t)d->N;
+    sp.nblk = (int32_t)((d->Sq + kBlockM - 1) / kBlockM);
+    if ((int64_t)sp.B * sp.N * sp.nblk != h->n_items)
+      return fail(FA_ERR_DEVICE, "internal: dense-mask work list has %d items, expected %lld",
+                  h->n_items, (long long)sp.B * sp.N * sp.nblk);
+    // The list, item_tr and the pre-pass's table are rewritten every call:
+    // a kernel of this handle on another stream may still be reading them.
+    if (h->any_call) {
+      cudaError_t e = cudaStreamWaitEvent(stream, h->last_call, 0);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+    }
+    if (ranges != nullptr) {
+      a.ranges = reinterpret_cast<TileRange*>(const_cast<int32_t*>(ranges));
+    } else {
+      occupancy_bind(&a, ws + occupancy_offset(h->n_seqs, h->n_items));
+      cudaError_t e = launch_occupancy(a, h->num_sms, stream);
+      if (e != cudaSuccess) return cuda_fail(e, "occupancy pre-pass launch");
+    }
+    sp.ranges = a.ranges;
+    sp.items = const_cast<WorkItem*>(p.items);
+    sp.item_tr = reinterpret_cast<TileRange*>(ws + item_tr_offset(h->n_seqs, h->n_items));
+    sp.occ_sb = (d->mask_kind == FA_MASK_SS) ? 0 : (d->mask_kind == FA_MASK_B1SS ? 1 : d->N);
+    sp.occ_sh = (d->mask_kind == FA_MASK_BNSS) ? 1 : 0;
+    sp.n_qt = a.n_qt;
+    sp.sq = (int32_t)d->Sq;
+    sp.n_kt = a.n_kt;
+    cudaError_t e = launch_schedule(sp, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "work list schedule launch");
+    p.item_tr = sp.item_tr;
+  }
   p.n_items = h->n_items;
   p.tnd = d->layout == FA_TND ? 1 : 0;
   p.scale_log2 = (float)(d->scale * 1.4426950408889634073599);
@@ -304,6 +387,67 @@ fa_status_t fa_fwd(fa_handle_t h, const void* q, const void* k, const void* v,
   e = cudaEventRecord(h->last_call, stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   h->any_call = true;
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status_t fa_fwd(fa_handle_t h, const void* q, const void* k, const void* v,
+                   const uint8_t* atten_mask, const int64_t* prefix,
+                   const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen, void* o,
+                   float* lse, void* cuda_stream) {
+  clear_error();
+  return forward(h, q, k, v, atten_mask, nullptr, prefix, actual_seq_qlen, actual_seq_kvlen, o,
+                 lse, cuda_stream);
+}
+
+fa_status_t fa_fwd_with_ranges(fa_handle_t h, const void* q, const void* k, const void* v,
+                               const uint8_t* atten_mask, const int32_t* ranges, void* o,
+                               float* lse, void* cuda_stream) {
+  clear_error();
+  if (!h) return fail(FA_ERR_NULLPTR, "handle is NULL");
+  if (h->desc.sparse_mode > 1 || h->desc.mask_kind == FA_MASK_NONE || !atten_mask)
+    return fail(FA_ERR_PARAM_INVALID,
+                "fa_fwd_with_ranges needs sparse_mode 0 or 1 with a mask kind and atten_mask");
+  if (!ranges) return fail(FA_ERR_NULLPTR, "ranges is NULL");
+  if ((uintptr_t)ranges & 15u) return fail(FA_ERR_PARAM_INVALID, "ranges must be 16-byte aligned");
+  return forward(h, q, k, v, atten_mask, ranges, nullptr, nullptr, nullptr, o, lse, cuda_stream);
+}
+
+fa_status_t fa_mask_occupancy(const fa_desc_t* desc, const uint8_t* atten_mask,
+                              uint8_t* tile_class, int32_t* ranges, void* cuda_stream) {
+  clear_error();
+  if (!desc) return fail(FA_ERR_NULLPTR, "desc is NULL");
+  if (!atten_mask || !tile_class || !ranges)
+    return fail(FA_ERR_NULLPTR, "atten_mask, tile_class and ranges are required");
+  fa_status_t st = validate_desc(desc);
+  if (st != FA_OK) return st;
+  if (desc->sparse_mode > 1 || desc->mask_kind == FA_MASK_NONE)
+    return fail(FA_ERR_PARAM_INVALID, "the occupancy pre-pass needs sparse_mode 0 or 1 with a mask");
+  st = validate_call(desc, nullptr, nullptr, nullptr, 1);
+  if (st != FA_OK) return st;
+  if ((uintptr_t)ranges & 15u) return fail(FA_ERR_PARAM_INVALID, "ranges must be 16-byte aligned");
+  int dev = 0, major = 0, minor = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  if (major != 10 || minor != 0)
+    return fail(FA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library runs on sm_100 (B200)", dev,
+                major, minor);
+  std::vector<SeqRec> recs = decode_geometry(desc, nullptr, nullptr, nullptr, 1);
+  if (recs.empty()) return FA_OK;
+  OccParams a;
+  std::memset(&a, 0, sizeof(a));
+  occupancy_shape(&a, recs[0], mask_planes(desc, 1));
+  a.mask = atten_mask;
+  a.cls = tile_class;
+  a.ranges = reinterpret_cast<TileRange*>(ranges);
+  e = launch_occupancy(a, sms, static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) return cuda_fail(e, "occupancy pre-pass launch");
   return FA_OK;
 }
 

@@ -30,6 +30,9 @@ struct __align__(64) FwdParams {
   int64_t o_sb, o_sh, o_st;  // O element strides: batch, head, token
   int64_t l_sb, l_sh;        // lse element strides: batch, head (token stride 1)
   int64_t m_sb, m_sh, m_si;  // mask element strides: batch, head, row (column stride 1)
+  // Dense-mask calls (or null): the key-tile ranges of sub-tiles 0 and 1
+  // of work item idx are item_tr[2 idx] and item_tr[2 idx + 1].
+  const TileRange* item_tr;
   int32_t n_items;
   int32_t tnd;             // packed tokens: TMA batch coordinate 0, token = offset + row
   float scale_log2;        // scale * log2(e)
@@ -42,6 +45,48 @@ enum DebugFlags : uint32_t {
   // wait on it runs out: exercises the bounded-wait abort path.
   kDebugDropFirstQ = 1u,
 };
+
+// Dense-mask tile occupancy (sparseMode 0 with an attenMask, sparseMode 1).
+// Pass 1 classifies every 128 x 128 tile of every mask plane as EMPTY (no
+// visible pair), FULL (every stored row sees all 128 keys) or PARTIAL; pass
+// 2 reduces each plane's row of tiles (one 128-row query sub-tile) to the
+// TileRange the attention kernel walks.
+struct OccParams {
+  const uint8_t* mask;   // planes of Sq x Skv bytes, nonzero = masked
+  uint8_t* cls;          // out: [plane][qt][kt] tile classes (fa_tile_class_t values)
+  TileRange* ranges;     // out: [plane][qt]
+  SeqRec geo;            // the geometry every sequence shares (BNSD/BSND)
+  int64_t m_plane;       // bytes per mask plane (Sq * Skv)
+  int64_t n_planes;
+  int32_t n_qt, n_kt;    // 128-row query sub-tiles, 128-key tiles
+  int32_t vec16;         // mask base and rows 16-byte aligned: 16-byte loads
+};
+
+// Scratch bytes of the pre-pass for `n_planes` planes of Sq x Skv: the
+// ranges (16 bytes per sub-tile, rounded up to 256) then the classes.
+size_t occupancy_bytes(int64_t n_planes, int64_t sq, int64_t skv);
+// Fill the pointer-free fields of `a` (the caller sets mask, cls, ranges).
+void occupancy_shape(OccParams* a, const SeqRec& geo, int64_t n_planes);
+// Enqueue both passes on `stream`.
+cudaError_t launch_occupancy(const OccParams& a, int num_sms, cudaStream_t stream);
+
+// The work list of a dense-mask call (BNSD/BSND: items (b, block of 256
+// rows, h) for every b, block and h), rebuilt on the device from the
+// pre-pass's ranges: longest first by the real key-tile count (ties in the
+// host list's (b, block, h) order), each item's two sub-tile ranges beside
+// it in item_tr. Lists longer than kSortMaxItems keep the (b, block, h)
+// order.
+struct SchedParams {
+  const TileRange* ranges;  // [plane][qt] from the pre-pass
+  WorkItem* items;          // out: [n]
+  TileRange* item_tr;       // out: [2 n]
+  int64_t occ_sb, occ_sh;   // plane = b * occ_sb + h * occ_sh
+  int32_t B, N, nblk;       // items = B * nblk * N
+  int32_t n_qt, sq;         // 128-row sub-tiles per plane, query rows
+  int32_t n_kt;             // key tiles (a sub-tile's cost is at most n_kt)
+};
+constexpr int64_t kSortMaxItems = 65536;  // 2 bytes each in shared memory
+cudaError_t launch_schedule(const SchedParams& s, cudaStream_t stream);
 
 // Build a 4-D bf16 tensor map over (D, S, N, B) with the given element
 // strides of S, N and B, boxes of 64 x 128 x 1 x 1, 128-byte swizzle.

@@ -415,15 +415,35 @@ struct ItemPlan {
   int nsub;        // sub-tiles with at least one stored row
 };
 
-__device__ __forceinline__ ItemPlan plan_item(const SeqRec& s, int qblk) {
+// Key-tile range of query sub-tile st of item it: the closed-form geometry,
+// or, for a dense attenMask, the range the occupancy pre-pass reduced the
+// mask to. Every role derives its tile sequence from this one function.
+// The kernel is compiled twice: kOcc (dense-mask calls whose pre-pass ran,
+// p.item_tr set) reads the ranges stored beside work item idx, the other
+// computes the closed form, so neither carries the other's code.
+template <bool kOcc>
+__device__ __forceinline__ TileRange sub_range(const FwdParams& p, int idx, const WorkItem& it,
+                                               const SeqRec& s, int st) {
+  if constexpr (kOcc) {
+    // item_tr is 256-byte aligned and 16 bytes per entry: one vector load.
+    const int4 v = __ldg(reinterpret_cast<const int4*>(p.item_tr) + 2 * (int64_t)idx + st);
+    return TileRange{v.x, v.y, v.z, v.w};
+  } else {
+    return tile_range(s, (int64_t)it.qblk * kBlockM + st * kTileM);
+  }
+}
+
+template <bool kOcc>
+__device__ __forceinline__ ItemPlan plan_item(const FwdParams& p, int idx, const WorkItem& it,
+                                              const SeqRec& s) {
   ItemPlan ip;
   ip.lo = 0x7fffffff;
   ip.hi = 0;
   ip.nsub = 0;
 #pragma unroll
   for (int st = 0; st < 2; ++st) {
-    const int64_t r0 = (int64_t)qblk * kBlockM + st * kTileM;
-    ip.tr[st] = tile_range(s, r0);
+    const int64_t r0 = (int64_t)it.qblk * kBlockM + st * kTileM;
+    ip.tr[st] = sub_range<kOcc>(p, idx, it, s, st);
     if (r0 < s.sq) ip.nsub = st + 1;
     if (ip.tr[st].hi > ip.tr[st].lo) {
       ip.lo = min(ip.lo, ip.tr[st].lo);
@@ -447,7 +467,7 @@ __device__ __forceinline__ bool active(const TileRange& t, int j) { return j >= 
 // first K (or the end of the work list). A Q tile is loaded once its buffer
 // is released by the last QK of the previous item on that sub-tile; placing
 // Q1 after the first K keeps a late Q1 release from holding back K.
-template <int D>
+template <int D, bool kOcc>
 __device__ void load_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint8_t* sQ,
                           uint8_t* sKV, const WaitCtx& w) {
   using C = Cfg<D>;
@@ -491,7 +511,7 @@ __device__ void load_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint8_t
     if (idx >= p.n_items) break;
     const WorkItem it = p.items[idx];
     const SeqRec sr = p.seqs[it.b];
-    const ItemPlan ip = plan_item(sr, it.qblk);
+    const ItemPlan ip = plan_item<kOcc>(p, idx, it, sr);
     if (ip.hi <= ip.lo) continue;
     const int bc = p.tnd ? 0 : it.b;
     if (ip.tr[0].hi > ip.tr[0].lo) ok = load_q(it, sr, 0, bc);
@@ -571,12 +591,13 @@ struct MmaPlan {
 };
 
 // Next item of this CTA with at least one key tile, from position k on.
+template <bool kOcc>
 __device__ __forceinline__ bool next_item(const FwdParams& p, int& k, MmaPlan& mp) {
   for (;; ++k) {
     const int idx = item_index(k);
     if (idx >= p.n_items) return false;
     const WorkItem it = p.items[idx];
-    const ItemPlan ip = plan_item(p.seqs[it.b], it.qblk);
+    const ItemPlan ip = plan_item<kOcc>(p, idx, it, p.seqs[it.b]);
     if (ip.hi > ip.lo) {
       mp.pos = k;
       ++k;
@@ -610,7 +631,7 @@ __device__ __forceinline__ uint32_t ring_v(uint32_t g, bool last) {
 // It runs ahead of the P.V stream (another thread), limited only by the
 // softmax releasing S, so the scores of the next tile, also across item
 // boundaries, are ready when the softmax wants them.
-template <int D>
+template <int D, bool kOcc>
 __device__ void qk_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t tmem,
                         const uint8_t* sQ, const uint8_t* sKV, const WaitCtx& w) {
   using C = Cfg<D>;
@@ -621,7 +642,7 @@ __device__ void qk_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
   bool ok = true;
   int k = 0;
   MmaPlan cur;
-  while (ok && next_item(p, k, cur)) {
+  while (ok && next_item<kOcc>(p, k, cur)) {
     bool q_ready[2] = {false, false};
     for (int t = cur.lo[2]; t < cur.hi[2] && ok; ++t, ++g) {
       const uint32_t r = ring_k(g);
@@ -665,7 +686,7 @@ __device__ void qk_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
 // the commit after it tells the softmax that O_s is updated and that the P
 // buffer may be rewritten. The first PV of an item overwrites O_s, so it
 // waits until the epilogue has read O_s of the previous item that had one.
-template <int D>
+template <int D, bool kOcc>
 __device__ void pv_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t tmem,
                         const uint8_t* sP, const uint8_t* sKV, const WaitCtx& w) {
   using C = Cfg<D>;
@@ -676,10 +697,10 @@ __device__ void pv_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
   bool ok = true;
   int k = 0;
   MmaPlan cur;
-  bool have = next_item(p, k, cur);
+  bool have = next_item<kOcc>(p, k, cur);
   while (ok && have) {
     MmaPlan nxt;
-    const bool have_next = next_item(p, k, nxt);
+    const bool have_next = next_item<kOcc>(p, k, nxt);
     bool first[2] = {true, true};
     for (int t = cur.lo[2]; t < cur.hi[2] && ok; ++t, ++g) {
       const uint32_t r = ring_v(g, !have_next && t + 1 == cur.hi[2]);
@@ -809,7 +830,7 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // warpgroup that does not visit the tile passes its turn on. At the end of
 // an item it writes the row's log-sum-exp and hands 1/l to the epilogue
 // warpgroup.
-template <int D>
+template <int D, bool kOcc>
 __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, float* inv_l_sm,
                              uint32_t tmem, uint8_t* sP, int sub, const WaitCtx& w) {
   using C = Cfg<D>;
@@ -822,6 +843,10 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
   const uint32_t tP = tmem + lane_bits + C::col_p(sub);
   const uint32_t sPs = smem_u32(sP) + sub * C::kPTileBytes;
   const float scale_log2 = p.scale_log2;
+  // Dense-mask rows start on 16-byte boundaries (base and row stride); the
+  // 16-byte gather below is compiled into the dense-mask variant only.
+  const bool mask_vec =
+      kOcc && ((reinterpret_cast<uintptr_t>(p.mask) | (uintptr_t)p.m_si) & 15u) == 0;
   uint32_t s_count = 0;   // S tiles consumed
   uint32_t pv_count = 0;  // P tiles produced = PV MMAs of this sub-tile
   uint32_t turn = 0;      // exponential-unit turns taken
@@ -833,9 +858,12 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
     const SeqRec sr = p.seqs[it.b];
     // The next item's record is read at the item boundary, on the critical
     // path of the exponential-unit turns: pull it into L1 now.
-    if (lane == 0 && item_index(k + 1) < p.n_items)
+    if (lane == 0 && item_index(k + 1) < p.n_items) {
       asm volatile("prefetch.global.L1 [%0];" ::"l"(p.items + item_index(k + 1)));
-    const ItemPlan ip = plan_item(sr, it.qblk);
+      if constexpr (kOcc)
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(p.item_tr + 2 * item_index(k + 1)));
+    }
+    const ItemPlan ip = plan_item<kOcc>(p, idx, it, sr);
     const TileRange tr = ip.tr[sub];
     const int64_t r0 = (int64_t)it.qblk * kBlockM + sub * kTileM;
     const int i = (int)(r0 + row);  // query row inside the sequence
@@ -851,6 +879,15 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
       mrow = p.mask + it.b * p.m_sb + it.h * p.m_sh + (int64_t)i * p.m_si;
     float m_used = -INFINITY;  // reference max (log2 units, scaled)
     float l = 0.f;             // running sum relative to m_used
+    // Dense-mask variant: the mask line of the next tile that needs it is
+    // pulled into L1 a tile ahead, so the gather after S arrives hits L1.
+    auto prefetch_mask = [&](int tn) {
+      if constexpr (kOcc) {
+        if (mrow != nullptr && tn >= tr.lo && tn < tr.hi && !(tn >= tr.full_lo && tn < tr.full_hi))
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(mrow + (int64_t)tn * kTileN));
+      }
+    };
+    prefetch_mask(tr.lo);
     for (int t = ip.lo; t < ip.hi; ++t) {
       // Turn on the exponential unit: warpgroup 0 goes first in every tile.
       uint64_t* my_turn = &ctl->mufu[sub];
@@ -868,6 +905,7 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
         if (lane == 0) arrive_token(&ctl->mufu[sub ^ 1], zero);
         continue;
       }
+      prefetch_mask(t + 1);
       if (!wait_warp(&ctl->s_full[sub], s_count & 1u, w, kSiteSFull)) {
         ok = false;
         break;
@@ -880,13 +918,36 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
       uint32_t mbits[4] = {0u, 0u, 0u, 0u};
       if (partial && mrow != nullptr) {
         const uint8_t* mt = mrow + (int64_t)t * kTileN;
+        bool vec = false;
+        if constexpr (kOcc) vec = mask_vec && (t + 1) * kTileN <= sr.skv;
+        if (vec) {
+          // The whole 128-byte tile row lies inside the mask row and is
+          // 16-byte aligned: eight 16-byte loads in flight at once, one bit
+          // per nonzero byte. Bits outside [c_lo, c_hi] are harmless, those
+          // keys are hidden by the window anyway.
+          uint4 v[8];
 #pragma unroll
-        for (int wd = 0; wd < 4; ++wd) {
-          uint32_t bits = 0u;
+          for (int q = 0; q < 8; ++q) v[q] = __ldg(reinterpret_cast<const uint4*>(mt) + q);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t wv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              const uint32_t e = __vcmpne4(wv[r], 0u);  // 0xff in every nonzero byte
+              const uint32_t nib =
+                  (e & 1u) | ((e >> 7) & 2u) | ((e >> 14) & 4u) | ((e >> 21) & 8u);
+              mbits[q >> 1] |= nib << (16 * (q & 1) + 4 * r);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int wd = 0; wd < 4; ++wd) {
+            uint32_t bits = 0u;
 #pragma unroll 1
-          for (int c = wd * 32; c < wd * 32 + 32; ++c)
-            if (c >= c_lo && c <= c_hi && mt[c] != 0) bits |= 1u << (c & 31);
-          mbits[wd] = bits;
+            for (int c = wd * 32; c < wd * 32 + 32; ++c)
+              if (c >= c_lo && c <= c_hi && mt[c] != 0) bits |= 1u << (c & 31);
+            mbits[wd] = bits;
+          }
         }
       }
       tc_fence_after();
@@ -976,7 +1037,7 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
 // item and sub-tile, once the softmax has handed over 1/l and the item's last
 // PV is done, O_s / l -> bf16 rows in global memory (zeros for rows that see
 // no key); 1/l is released as soon as it is read, O_s once it is read.
-template <int D>
+template <int D, bool kOcc>
 __device__ void epilogue_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl,
                               const float* inv_l_sm, uint32_t tmem, const WaitCtx& w) {
   using C = Cfg<D>;
@@ -992,7 +1053,7 @@ __device__ void epilogue_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl,
 #pragma unroll 1
     for (int sub = 0; sub < 2; ++sub) {
       const int64_t r0 = (int64_t)it.qblk * kBlockM + sub * kTileM;
-      const TileRange tr = tile_range(sr, r0);
+      const TileRange tr = sub_range<kOcc>(p, idx, it, sr, sub);
       const int i = (int)(r0 + row);
       const bool row_valid = i < sr.sq;
       if (!wait_warp(&ctl->epi_full[sub], k & 1u, w, kSiteEpi)) return;
@@ -1032,7 +1093,7 @@ __device__ void epilogue_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl,
   }
 }
 
-template <int D>
+template <int D, bool kOcc>
 __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100(const __grid_constant__ FwdParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -1087,15 +1148,15 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100(const __grid_constan
 
   if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-    softmax_role<D>(p, ctl, inv_l_sm, tmem, sP, warp >> 2, w);
+    softmax_role<D, kOcc>(p, ctl, inv_l_sm, tmem, sP, warp >> 2, w);
   } else if (warp < 12) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
-    epilogue_role<D>(p, ctl, inv_l_sm, tmem, w);
+    epilogue_role<D, kOcc>(p, ctl, inv_l_sm, tmem, w);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
-    if (warp == kWarpMma && lane == 0) qk_role<D>(p, ctl, tmem, sQ, sKV, w);
-    if (warp == kWarpPv && lane == 0) pv_role<D>(p, ctl, tmem, sP, sKV, w);
-    if (warp == kWarpLoad && lane == 0) load_role<D>(p, ctl, sQ, sKV, w);
+    if (warp == kWarpMma && lane == 0) qk_role<D, kOcc>(p, ctl, tmem, sQ, sKV, w);
+    if (warp == kWarpPv && lane == 0) pv_role<D, kOcc>(p, ctl, tmem, sP, sKV, w);
+    if (warp == kWarpLoad && lane == 0) load_role<D, kOcc>(p, ctl, sQ, sKV, w);
   }
   __syncwarp();
   tc_fence_before();
@@ -1145,10 +1206,10 @@ bool encode_operand_map(CUtensorMap* tm, const void* base, int64_t D, int64_t S,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool kOcc>
 static cudaError_t launch_d(const FwdParams& p, int grid, cudaStream_t stream, const char** why) {
   using C = dev::Cfg<D>;
-  auto kern = dev::fa_fwd_sm100<D>;
+  auto kern = dev::fa_fwd_sm100<D, kOcc>;
   static bool configured = false;
   static bool regs_ok = false;
   if (!configured) {
@@ -1173,8 +1234,11 @@ static cudaError_t launch_d(const FwdParams& p, int grid, cudaStream_t stream, c
 
 cudaError_t launch_fwd(int D, const FwdParams& p, int grid, cudaStream_t stream,
                        const char** why) {
-  if (D == 128) return launch_d<128>(p, grid, stream, why);
-  if (D == 64) return launch_d<64>(p, grid, stream, why);
+  const bool occ = p.item_tr != nullptr;
+  if (D == 128) return occ ? launch_d<128, true>(p, grid, stream, why)
+                           : launch_d<128, false>(p, grid, stream, why);
+  if (D == 64) return occ ? launch_d<64, true>(p, grid, stream, why)
+                          : launch_d<64, false>(p, grid, stream, why);
   if (why) *why = "unsupported head dim";
   return cudaErrorInvalidValue;
 }

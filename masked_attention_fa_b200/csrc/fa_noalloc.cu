@@ -16,6 +16,13 @@
 //     256 bytes) and the work list (16 bytes per (sequence, head, block of
 //     256 query rows)). Larger problems are rejected with FA_ERR_UNSUPPORTED
 //     before any device work.
+//   - A dense-mask call (sparseMode 1, or 0 with an attenMask) also puts
+//     each work item's two key-tile ranges (32 bytes per item) and the
+//     occupancy pre-pass's scratch (16 bytes per mask plane and 128-row query
+//     sub-tile, rounded up to 256, plus 1 byte per plane and 128 x 128 tile)
+//     behind the work list when they fit; when they do not, the call still
+//     runs, without the pre-pass (every tile of the band is visited with the
+//     element mask), and gives the same result.
 //   - Every call, on every stream, shares the one array per device and leaves
 //     its own work list in it. Calls whose kernels overlap on the GPU (for
 //     example on two streams without ordering between them) race on the
@@ -260,6 +267,45 @@ extern "C" fa_status_t fa_fwd_noalloc(const fa_desc_t* desc, const void* q, cons
     p.m_si = d->Skv;
     p.m_sb = (d->mask_kind == FA_MASK_SS) ? 0 : (d->mask_kind == FA_MASK_B1SS ? plane : d->N * plane);
     p.m_sh = (d->mask_kind == FA_MASK_BNSS) ? plane : 0;
+  }
+  if (has_mask && n > 0) {
+    // The occupancy pre-pass and the device-side list rebuild run when their
+    // scratch (each item's ranges, the pre-pass's table and classes) fits
+    // behind the work list; otherwise the kernel visits every tile of the
+    // band with the element mask, which gives the same result more slowly.
+    const int64_t planes = d->mask_kind == FA_MASK_SS ? 1
+                           : d->mask_kind == FA_MASK_B1SS ? d->B
+                                                          : d->B * d->N;
+    const size_t tr_off = round256(need);
+    const size_t occ_off = tr_off + round256(n * 2 * sizeof(TileRange));
+    if (occ_off + occupancy_bytes(planes, d->Sq, d->Skv) <= kNoAllocScratchBytes) {
+      OccParams a;
+      std::memset(&a, 0, sizeof(a));
+      occupancy_shape(&a, recs[0], planes);
+      a.mask = atten_mask;
+      a.ranges = reinterpret_cast<TileRange*>(dscr + occ_off);
+      a.cls = dscr + occ_off + round256((size_t)(planes * a.n_qt) * sizeof(TileRange));
+      e = launch_occupancy(a, slot->num_sms, stream);
+      if (e != cudaSuccess) return cuda_err(e, "occupancy pre-pass launch");
+      SchedParams sp;
+      std::memset(&sp, 0, sizeof(sp));
+      sp.ranges = a.ranges;
+      sp.items = reinterpret_cast<WorkItem*>(dscr + kNoAllocHeaderBytes + seq_bytes);
+      sp.item_tr = reinterpret_cast<TileRange*>(dscr + tr_off);
+      sp.occ_sb = (d->mask_kind == FA_MASK_SS) ? 0 : (d->mask_kind == FA_MASK_B1SS ? 1 : d->N);
+      sp.occ_sh = (d->mask_kind == FA_MASK_BNSS) ? 1 : 0;
+      sp.B = (int32_t)d->B;
+      sp.N = (int32_t)d->N;
+      sp.nblk = (int32_t)((d->Sq + kBlockM - 1) / kBlockM);
+      sp.n_qt = a.n_qt;
+      sp.sq = (int32_t)d->Sq;
+      sp.n_kt = a.n_kt;
+      if ((size_t)sp.B * sp.N * sp.nblk != n)
+        return fail(FA_ERR_DEVICE, "internal: dense-mask work list has %zu items", n);
+      e = launch_schedule(sp, stream);
+      if (e != cudaSuccess) return cuda_err(e, "work list schedule launch");
+      p.item_tr = sp.item_tr;
+    }
   }
   p.n_items = (int32_t)n;
   p.tnd = tnd ? 1 : 0;

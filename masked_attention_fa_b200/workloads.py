@@ -9,9 +9,10 @@ workload's seed draws, in this order, the varlen lengths (TND workloads
 only), then q, k and v as float32 N(0, 1) which are rounded to bfloat16.
 The scale is 1/sqrt(D).
 
-The five named workloads follow the shapes of the Ascend "sparseMode参数说明"
+The named workloads follow the shapes of the Ascend "sparseMode参数说明"
 page's scenarios (band, leftUpCausal, right-down band, varlen
-rightDownCausal, prefix) at sizes of long-context inference.
+rightDownCausal, prefix, and the causal case given as an explicit allMask)
+at sizes of long-context inference.
 """
 from __future__ import annotations
 
@@ -103,8 +104,53 @@ def lower_triangular_mask(S: int) -> torch.Tensor:
     return torch.triu(torch.ones(S, S, dtype=torch.uint8), diagonal=1)
 
 
+# Patterns of block_mask, one per 128 x 128 block (1 = masked).
+BLOCK_PATTERNS = ("hidden", "visible", "random", "one_visible", "one_hidden", "lower")
+
+
+def block_mask(shape, seed: int, block: int = 128, weights=None) -> torch.Tensor:
+    """A uint8 mask of `shape` (..., Sq, Skv) made of blocks of `block` rows x
+    `block` keys, each drawn from BLOCK_PATTERNS with the given weights (by
+    default: hidden 0.35, visible 0.3, random 0.15, one visible / one hidden
+    pair 0.05 each, lower triangle 0.1): whole hidden and whole visible blocks
+    as in the page's causal and band masks, and mixed ones. Leading dims are
+    independent planes."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    w = torch.tensor(weights or [0.35, 0.3, 0.15, 0.05, 0.05, 0.1], dtype=torch.float64)
+    *lead, Sq, Skv = shape
+    nq, nk = (Sq + block - 1) // block, (Skv + block - 1) // block
+    planes = 1
+    for d in lead:
+        planes *= d
+    out = torch.ones((planes, nq * block, nk * block), dtype=torch.uint8)
+    pat = torch.multinomial(w, planes * nq * nk, replacement=True, generator=g)
+    rnd = (torch.rand((planes, nq * block, nk * block), generator=g) < 0.3).to(torch.uint8)
+    pos = torch.randint(0, block * block, (planes * nq * nk,), generator=g)
+    tri = torch.triu(torch.ones(block, block, dtype=torch.uint8), diagonal=1)
+    n = 0
+    for p in range(planes):
+        for a in range(nq):
+            for b in range(nk):
+                blk = out[p, a * block:(a + 1) * block, b * block:(b + 1) * block]
+                kind = BLOCK_PATTERNS[int(pat[n])]
+                r, c = divmod(int(pos[n]), block)
+                if kind == "visible":
+                    blk.zero_()
+                elif kind == "random":
+                    blk.copy_(rnd[p, a * block:(a + 1) * block, b * block:(b + 1) * block])
+                elif kind == "one_visible":
+                    blk[r, c] = 0
+                elif kind == "one_hidden":
+                    blk.zero_()
+                    blk[r, c] = 1
+                elif kind == "lower":
+                    blk.copy_(tri)
+                n += 1
+    return out[:, :Sq, :Skv].reshape(*lead, Sq, Skv).contiguous()
+
+
 def named_workloads() -> dict:
-    """The five long-context scenarios, by name."""
+    """The long-context scenarios, by name."""
     g4 = torch.Generator("cpu").manual_seed(4)
     cu_q, cu_kv = varlen_lengths(g4, 16, 512, 4096, 1024)
     return {
@@ -121,6 +167,10 @@ def named_workloads() -> dict:
                                            actual_seq_kvlen=cu_kv),
         "prefix_8k": Workload("prefix_8k", "BNSD", 4, 16, 8192, 8192, 128, 5, seed=5,
                               prefix=[512, 1024, 2048, 4096]),
+        # the leftUpCausal problem (same shape and seed, so the same q, k, v)
+        # given as an explicit lower-triangular allMask (sparseMode 1)
+        "allmask_causal_4k": Workload("allmask_causal_4k", "BNSD", 2, 16, 4096, 4096, 128, 1,
+                                      seed=2, mask_kind="SS"),
     }
 
 
@@ -139,7 +189,7 @@ def make_inputs(w: Workload, device="cpu"):
     v = torch.randn(w.kv_shape(), generator=g, dtype=torch.float32).to(torch.bfloat16)
     mask = None
     if w.mask_kind is not None:
-        if w.name == "band_causal_256":
+        if w.name in ("band_causal_256", "allmask_causal_4k"):
             mask = lower_triangular_mask(w.Sq)
         else:
             mask = (torch.rand(w.mask_shape(), generator=g) < 0.3).to(torch.uint8)

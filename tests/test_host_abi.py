@@ -266,3 +266,45 @@ def test_plan_stats_item_count_and_named_workload_counts():
     S = 8192
     expect = 16 * sum(P * P + S * (S + 1) // 2 - P * (P + 1) // 2 for P in w.prefix)
     assert fa.fa_visible_pairs(d, prefix=w.prefix) == expect == 2325942272
+
+
+def test_occupancy_entry_points_validate_before_device_work():
+    """fa_mask_occupancy and fa_fwd_with_ranges reject bad arguments on the
+    host, before any device query (the pointers below are never touched)."""
+    import ctypes
+    lib = fa.load_library()
+    dev = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10004)
+    ss1 = fa.make_desc("BNSD", 1, 1, 256, 256, 64, 1, mask_kind="SS")
+    causal = fa.make_desc("BNSD", 1, 1, 256, 256, 64, 2)
+    tnd = fa.make_desc("TND", 1, 1, 256, 256, 64, 1, mask_kind="SS")
+    occ = lib.fa_mask_occupancy
+    assert fa.STATUS[occ(ctypes.byref(ss1), None, dev, dev, None)] == "FA_ERR_NULLPTR"
+    assert fa.STATUS[occ(ctypes.byref(ss1), dev, dev, None, None)] == "FA_ERR_NULLPTR"
+    assert fa.STATUS[occ(ctypes.byref(causal), dev, dev, dev, None)] == "FA_ERR_PARAM_INVALID"
+    assert fa.STATUS[occ(ctypes.byref(tnd), dev, dev, dev, None)] == "FA_ERR_UNSUPPORTED"
+    assert fa.STATUS[occ(ctypes.byref(ss1), dev, dev, odd, None)] == "FA_ERR_PARAM_INVALID"
+    assert "16-byte" in fa.fa_last_error()
+    h1, h2 = fa.fa_create(ss1), fa.fa_create(causal)
+    try:
+        fwr = lib.fa_fwd_with_ranges
+        assert fa.STATUS[fwr(h2, dev, dev, dev, dev, dev, dev, dev, None)] == \
+            "FA_ERR_PARAM_INVALID"
+        assert fa.STATUS[fwr(h1, dev, dev, dev, None, dev, dev, dev, None)] == \
+            "FA_ERR_PARAM_INVALID"
+        assert fa.STATUS[fwr(h1, dev, dev, dev, dev, None, dev, dev, None)] == "FA_ERR_NULLPTR"
+        assert fa.STATUS[fwr(h1, dev, dev, dev, dev, odd, dev, dev, None)] == \
+            "FA_ERR_PARAM_INVALID"
+        assert fa.STATUS[fwr(None, dev, dev, dev, dev, dev, dev, dev, None)] == "FA_ERR_NULLPTR"
+    finally:
+        fa.fa_destroy(h1)
+        fa.fa_destroy(h2)
+
+
+def test_occupancy_output_shapes():
+    d = fa.make_desc("BSND", 3, 5, 300, 1000, 128, 0, 10, 10, None, "BNSS")
+    assert fa.occupancy_shapes(d) == ((15, 3, 8), (15, 3, 4))
+    d = fa.make_desc("BNSD", 3, 5, 128, 129, 128, 1, mask_kind="B1SS")
+    assert fa.occupancy_shapes(d) == ((3, 1, 2), (3, 1, 4))
+    d = fa.make_desc("BNSD", 3, 5, 1, 1, 64, 1, mask_kind="SS")
+    assert fa.occupancy_shapes(d) == ((1, 1, 1), (1, 1, 4))
