@@ -742,8 +742,9 @@ __device__ void pv_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
 
 // Scores of this thread's row (128 keys of S_s) with the element mask of a
 // boundary tile applied (-inf where the key is not visible). The visible
-// columns [c_lo, c_hi] are tested as one unsigned range compare per element;
-// dense-mask bits (modes 0/1) are applied only when present.
+// columns [c_lo, c_hi] and, for a dense mask, its bits become four words of
+// one bit per key, and each score is kept or replaced by one bit test (a
+// quarter of the cost of a range compare per key, measured).
 __device__ __forceinline__ void load_scores(uint32_t tS, float (&x)[128], bool partial, int c_lo,
                                             int c_hi, bool dense, const uint32_t (&mbits)[4]) {
   uint32_t sv[128];
@@ -751,16 +752,18 @@ __device__ __forceinline__ void load_scores(uint32_t tS, float (&x)[128], bool p
 #pragma unroll
   for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sv[c]);
   if (partial) {
-    int lo = c_lo, width = c_hi - c_lo;
-    if (width < 0) lo = 1 << 20, width = 0;  // nothing visible
+    // One bit per key: visible = inside [c_lo, c_hi] and (dense) unmasked.
+    uint32_t wm[4];
+#pragma unroll
+    for (int wd = 0; wd < 4; ++wd) {
+      const int a = c_lo - 32 * wd, b = c_hi - 32 * wd;  // visible bits [a, b] of this word
+      const uint32_t upto = b >= 31 ? 0xffffffffu : (b < 0 ? 0u : (0xffffffffu >> (31 - b)));
+      const uint32_t from = a <= 0 ? 0xffffffffu : (a > 31 ? 0u : (0xffffffffu << a));
+      wm[wd] = upto & from & ~(dense ? mbits[wd] : 0u);
+    }
 #pragma unroll
     for (int c = 0; c < 128; ++c)
-      x[c] = ((unsigned)(c - lo) <= (unsigned)width) ? x[c] : -INFINITY;
-    if (dense) {
-#pragma unroll
-      for (int c = 0; c < 128; ++c)
-        x[c] = ((mbits[c >> 5] >> (c & 31)) & 1u) ? -INFINITY : x[c];
-    }
+      x[c] = ((wm[c >> 5] >> (c & 31)) & 1u) ? x[c] : -INFINITY;
   }
 }
 
@@ -976,14 +979,25 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       // The other warpgroup gets its turn once the first kTokenCol keys are
       // done, so both feed the exponential unit across the handover.
-      if (partial) exp_pack_part<false, 0, kTokenCol>(x, m2, c2, acc, pk);
-      else exp_pack_part<true, 0, kTokenCol>(x, m2, c2, acc, pk);
+      // One instance of the exponential loop serves every tile while the
+      // FMA-pipe polynomial is off: a second copy for the (rarer) boundary
+      // tiles is cold in the instruction cache each time it runs.
+      if constexpr (kPolyPer8 > 0) {
+        if (partial) exp_pack_part<false, 0, kTokenCol>(x, m2, c2, acc, pk);
+        else exp_pack_part<true, 0, kTokenCol>(x, m2, c2, acc, pk);
+      } else {
+        exp_pack_part<false, 0, kTokenCol>(x, m2, c2, acc, pk);
+      }
       __syncwarp();
       if (lane == 0)
         arrive_token(&ctl->mufu[sub ^ 1], ((acc[0] + acc[1]) + (acc[2] + acc[3])) +
                                               ((acc[4] + acc[5]) + (acc[6] + acc[7])));
-      if (partial) exp_pack_part<false, kTokenCol, 128>(x, m2, c2, acc, pk);
-      else exp_pack_part<true, kTokenCol, 128>(x, m2, c2, acc, pk);
+      if constexpr (kPolyPer8 > 0) {
+        if (partial) exp_pack_part<false, kTokenCol, 128>(x, m2, c2, acc, pk);
+        else exp_pack_part<true, kTokenCol, 128>(x, m2, c2, acc, pk);
+      } else {
+        exp_pack_part<false, kTokenCol, 128>(x, m2, c2, acc, pk);
+      }
       l += sum_acc(acc);
       if (pv_count > 0) {
         // The previous PV of this sub-tile must be done: it still reads the
