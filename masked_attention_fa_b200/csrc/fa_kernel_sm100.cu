@@ -796,6 +796,19 @@ __device__ __forceinline__ float sum_acc(float (&acc)[8]) {
   return acc[0] + acc[1];
 }
 
+// O and lse stores that do not allocate in L1. The SM keeps only ~28 KB of
+// L1 beside 227 KB of shared memory; 64 KB of O per item written through it
+// evicts the work-item and sequence records every role reads at the next
+// item boundary (measured: +5 % causal, +2 % on the other workloads).
+__device__ __forceinline__ void st_global_na_v4(void* ptr, const uint4& v) {
+  asm volatile("st.global.L1::no_allocate.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(ptr), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_global_na_f32(float* ptr, float v) {
+  asm volatile("st.global.L1::no_allocate.f32 [%0], %1;" ::"l"(ptr), "f"(v) : "memory");
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
@@ -1042,7 +1055,7 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
     mbar_arrive(&ctl->epi_full[sub]);
     if (row_valid) {
       const float lse = l > 0.f ? (m_used + lg2_fast(l)) * 0.69314718055994530942f : -INFINITY;
-      p.lse[it.b * p.l_sb + it.h * p.l_sh + sr.q_off + i] = lse;
+      st_global_na_f32(p.lse + it.b * p.l_sb + it.h * p.l_sh + sr.q_off + i, lse);
     }
   }
 }
@@ -1093,7 +1106,7 @@ __device__ void epilogue_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl,
           if (row_valid) {
             uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = pkd[v];
+            for (int v = 0; v < 4; ++v) st_global_na_v4(dst + v, pkd[v]);
           }
         }
         tc_fence_before();
@@ -1101,7 +1114,7 @@ __device__ void epilogue_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl,
       } else if (row_valid) {
         uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll 1
-        for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+        for (int v = 0; v < D / 8; ++v) st_global_na_v4(dst + v, make_uint4(0u, 0u, 0u, 0u));
       }
     }
   }
