@@ -76,6 +76,9 @@ def _load():
         lib.oracle_tile_classes.restype = None
         lib.oracle_tile_ranges.argtypes = [P, i64, i64, P]
         lib.oracle_tile_ranges.restype = None
+        lib.oracle_attn_paged.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, P, P, P, i64, i64,
+                                          P, P]
+        lib.oracle_attn_paged.restype = ctypes.c_int
         lib.oracle_visible_count.argtypes = [ctypes.POINTER(_Desc), P, P, P, P]
         lib.oracle_visible_count.restype = ctypes.c_int64
         lib.oracle_flash_tiled.argtypes = [P, P, P, P, i64, i64, i64, i64, ctypes.c_double, P]
@@ -221,6 +224,26 @@ def attention(pb: Problem, q, k, v):
                               v.ctypes.data, o.ctypes.data, lse.ctypes.data)
     if err:
         raise MemoryError("oracle_attn: allocation failed")
+    return o, lse
+
+
+def attention_paged(pb: Problem, q, k_cache, v_cache, block_table, block_size: int):
+    """Forward of a TND problem with K/V read from paged caches
+    [num_blocks, block_size, N, D] through block_table [B, max_blocks]
+    (int32): returns (O [T_q, N, D], lse [N, T_q])."""
+    assert pb.layout == "TND"
+    q, kc, vc = _f64(q), _f64(k_cache), _f64(v_cache)
+    bt = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+    assert q.shape == pb.q_shape() and kc.shape == vc.shape and kc.shape[1] == block_size
+    o = np.zeros(pb.q_shape(), dtype=np.float64)
+    lse = np.full(pb.lse_shape(), -np.inf, dtype=np.float64)
+    d = pb.desc()
+    pre, cq, ckv, _ = pb._ptrs()
+    err = _load().oracle_attn_paged(ctypes.byref(d), pre, cq, ckv, q.ctypes.data, kc.ctypes.data,
+                                    vc.ctypes.data, bt.ctypes.data, bt.shape[1], block_size,
+                                    o.ctypes.data, lse.ctypes.data)
+    if err:
+        raise MemoryError("oracle_attn_paged: allocation failed")
     return o, lse
 
 

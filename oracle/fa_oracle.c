@@ -21,6 +21,9 @@
  *     range of key blocks each query block must visit: the sparseMode page
  *     has the operator compute only the part the mask and the band leave
  *     visible, and these are that statement summarised by block.
+ *   - The same forward with keys and values read from paged caches (the
+ *     "Norm" layout of the aclnnScatterPaKvCache page, scenario 2) through
+ *     a per-sequence block table.
  *   - The tiled online-softmax recurrence (running max m_i, running sum l_i,
  *     normalised output) of the "FlashAttention tiling & online softmax"
  *     exercise page (section "Mục tiêu kiến thức"), used only to pin the
@@ -318,6 +321,86 @@ int oracle_attn_rows(const oracle_desc* d, const int64_t* prefix,
                    lse_rows + r);
         free(vis);
         free(scores);
+    }
+    return err;
+}
+
+/*
+ * Key or value row of logical key j of sequence b, head h, in a paged cache
+ * laid out as [num_blocks, block_size, N, D], the "Norm" cache of the
+ * aclnnScatterPaKvCache page (scenario 2). A token is written to slot
+ * block * block_size + offset; sequence b's key j sits in block
+ * block_table[b][j / block_size] at offset j % block_size.
+ */
+static const double* paged_row(const double* cache, const int32_t* block_table,
+                               int64_t max_blocks, int64_t block_size,
+                               int64_t N, int64_t D, int64_t b, int64_t h,
+                               int64_t j) {
+    const int64_t blk = block_table[b * max_blocks + j / block_size];
+    const int64_t slot = blk * block_size + j % block_size;
+    return cache + (slot * N + h) * D;
+}
+
+/*
+ * Forward with the keys and values read from paged caches instead of packed
+ * TND tensors. q, o: [T_q, N, D] (TND); lse: [N, T_q]; the visibility rule,
+ * the lengths (cumulative cu_q / cu_kv) and the plain softmax are those of
+ * oracle_attn; only where key j of sequence b is stored differs.
+ */
+int oracle_attn_paged(const oracle_desc* d, const int64_t* prefix,
+                      const int64_t* cu_q, const int64_t* cu_kv,
+                      const double* q, const double* k_cache,
+                      const double* v_cache, const int32_t* block_table,
+                      int64_t max_blocks, int64_t block_size, double* o,
+                      double* lse) {
+    int err = 0;
+    const int64_t nb = d->B, nh = d->N, D = d->D;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int64_t b = 0; b < nb; ++b) {
+        for (int64_t h = 0; h < nh; ++h) {
+            seq_info s = seq_of(d, cu_q, cu_kv, b);
+            int64_t skv_alloc = s.skv > 0 ? s.skv : 1;
+            double* scores = (double*)malloc(sizeof(double) * skv_alloc);
+            if (!scores) {
+#pragma omp atomic write
+                err = 1;
+                continue;
+            }
+            for (int64_t i = 0; i < s.sq; ++i) {
+                const double* qi = q + row_offset(d, d->Sq, b, h, s.q_off + i);
+                double* oi = o + row_offset(d, d->Sq, b, h, s.q_off + i);
+                double m = -INFINITY;
+                for (int64_t j = 0; j < s.skv; ++j) {
+                    scores[j] = -INFINITY;
+                    if (!oracle_visible(d, prefix, cu_q, cu_kv, NULL, b, h, i, j))
+                        continue;
+                    const double* kj = paged_row(k_cache, block_table, max_blocks,
+                                                 block_size, nh, D, b, h, j);
+                    double acc = 0.0;
+                    for (int64_t x = 0; x < D; ++x) acc += qi[x] * kj[x];
+                    scores[j] = d->scale * acc;
+                    if (scores[j] > m) m = scores[j];
+                }
+                for (int64_t x = 0; x < D; ++x) oi[x] = 0.0;
+                double* li = lse + lse_offset(d, b, h, s.q_off + i);
+                if (m == -INFINITY) {
+                    *li = -INFINITY;
+                    continue;
+                }
+                double l = 0.0;
+                for (int64_t j = 0; j < s.skv; ++j) {
+                    if (scores[j] == -INFINITY) continue;
+                    const double p = exp(scores[j] - m);
+                    l += p;
+                    const double* vj = paged_row(v_cache, block_table, max_blocks,
+                                                 block_size, nh, D, b, h, j);
+                    for (int64_t x = 0; x < D; ++x) oi[x] += p * vj[x];
+                }
+                for (int64_t x = 0; x < D; ++x) oi[x] /= l;
+                *li = m + log(l);
+            }
+            free(scores);
+        }
     }
     return err;
 }

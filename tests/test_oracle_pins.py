@@ -557,3 +557,83 @@ def test_tile_classes_match_bruteforce_blocks():
                 blk = pad[qt * t:min((qt + 1) * t, Sq), kt * t:(kt + 1) * t]
                 cls = 2 if blk.all() else (1 if blk.any() else 0)
                 assert got[qt, kt] == cls, (mode, qt, kt)
+
+
+# --------------------------------------------------------------------------
+# Paged K/V caches ("Norm" layout of the aclnnScatterPaKvCache page): key j
+# of sequence b sits at block block_table[b][j // bs], offset j % bs.
+# --------------------------------------------------------------------------
+
+def _paged_from_packed(k, v, cu_kv, bs, rng, spare=3, shuffle=True):
+    """Scatter packed TND K/V [T_kv, N, D] into caches of bs-token blocks in a
+    random block order; unused slots hold NaN so that reading one shows."""
+    T, N, D = k.shape
+    lens = np.diff(np.concatenate([[0], cu_kv]))
+    nblk = [(-(-int(n) // bs)) for n in lens]
+    total = sum(nblk) + spare
+    order = rng.permutation(total) if shuffle else np.arange(total)
+    kc = np.full((total, bs, N, D), np.nan)
+    vc = np.full((total, bs, N, D), np.nan)
+    table = np.full((len(lens), max(max(nblk), 1)), -1, dtype=np.int32)
+    nxt, start = 0, 0
+    for b, n in enumerate(lens):
+        for c in range(nblk[b]):
+            blk = int(order[nxt]); nxt += 1
+            table[b, c] = blk
+            rows = np.arange(c * bs, min((c + 1) * bs, n))
+            kc[blk, :len(rows)] = k[start + rows]
+            vc[blk, :len(rows)] = v[start + rows]
+        start += n
+    return kc, vc, table
+
+
+@pytest.mark.parametrize("mode,extra", [(3, {}), (2, {}), (0, {}), (4, dict(pre_tokens=5, next_tokens=1))])
+@pytest.mark.parametrize("bs", [4, 16])
+def test_paged_equals_packed_forward(mode, extra, bs):
+    """The paged forward with any block order equals the packed TND forward
+    (already pinned to SDPA and the page's examples), and never reads a slot
+    outside the sequences' keys (those hold NaN)."""
+    rng = np.random.default_rng(11)
+    lq, lkv = [1, 3, 0, 2], [7, 19, 5, 33]
+    cu_q, cu_kv = np.cumsum(lq).tolist(), np.cumsum(lkv).tolist()
+    N, D = 2, 8
+    q = rng.standard_normal((cu_q[-1], N, D))
+    k = rng.standard_normal((cu_kv[-1], N, D))
+    v = rng.standard_normal((cu_kv[-1], N, D))
+    pb = Problem("TND", len(lq), N, cu_q[-1], cu_kv[-1], D, sparse_mode=mode,
+                 actual_seq_qlen=cu_q, actual_seq_kvlen=cu_kv, **extra)
+    o_ref, l_ref = oracle.attention(pb, q, k, v)
+    for shuffle in (False, True):
+        kc, vc, table = _paged_from_packed(k, v, np.array(cu_kv), bs, rng, shuffle=shuffle)
+        o, l = oracle.attention_paged(pb, q, kc, vc, table, bs)
+        assert np.all(np.isfinite(o))
+        np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-13)
+        np.testing.assert_array_equal(np.isneginf(l), np.isneginf(l_ref))
+        live = ~np.isneginf(l_ref)
+        np.testing.assert_allclose(l[live], l_ref[live], rtol=0, atol=1e-13)
+
+
+def test_paged_decode_row_is_sdpa_over_the_gathered_keys():
+    """One decode row per sequence (rightDownCausal sees every key): torch
+    SDPA over the keys gathered by hand from the block table."""
+    rng = np.random.default_rng(12)
+    lkv = [9, 1, 40]
+    cu_q, cu_kv = [1, 2, 3], np.cumsum(lkv).tolist()
+    N, D, bs = 3, 16, 8
+    q = rng.standard_normal((3, N, D))
+    k = rng.standard_normal((cu_kv[-1], N, D))
+    v = rng.standard_normal((cu_kv[-1], N, D))
+    kc, vc, table = _paged_from_packed(k, v, np.array(cu_kv), bs, rng)
+    pb = Problem("TND", 3, N, 3, cu_kv[-1], D, sparse_mode=3, actual_seq_qlen=cu_q,
+                 actual_seq_kvlen=cu_kv)
+    o, l = oracle.attention_paged(pb, q, kc, vc, table, bs)
+    for b, n in enumerate(lkv):
+        idx = np.arange(n)
+        kb = kc[table[b, idx // bs], idx % bs]          # [n, N, D]
+        vb = vc[table[b, idx // bs], idx % bs]
+        qt = torch.from_numpy(q[b]).unsqueeze(1)           # [N, 1, D]
+        ref = _sdpa(qt, torch.from_numpy(kb).transpose(0, 1), torch.from_numpy(vb).transpose(0, 1),
+                    pb.scale).squeeze(1).numpy()
+        np.testing.assert_allclose(o[b], ref, rtol=0, atol=1e-12)
+        s = pb.scale * np.einsum("hd,nhd->hn", q[b], kb)
+        np.testing.assert_allclose(l[:, b], np.log(np.exp(s).sum(1)), rtol=0, atol=1e-12)
