@@ -197,6 +197,43 @@ fa_status_t fa_fwd_noalloc(const fa_desc_t* desc, const void* q, const void* k, 
                            void* o, float* lse, void* cuda_stream);
 
 /*
+ * fa_fwd_paged — forward of a TND handle with the keys and values read from
+ * paged caches instead of packed tensors, for decode-shaped calls (a few
+ * query rows per sequence against a long cached context).
+ *
+ * Cache layout: the "Norm" cache of the aclnnScatterPaKvCache page
+ * (scenario 2): k_cache and v_cache are device bf16 [num_blocks, block_size,
+ * N, D], a token written at slot s sitting in block s / block_size at offset
+ * s % block_size. Key j of sequence b is in block block_table[b][j /
+ * block_size] at offset j % block_size.
+ * q, o         device bf16 [T_q, N, D] (the handle's Sq = T_q), 16-byte aligned.
+ * lse          device fp32 [N, T_q], 4-byte aligned.
+ * block_table  device int32 [B, max_blocks], 4-byte aligned; only the first
+ *              ceil(Skv_b / block_size) entries of row b are read. An entry
+ *              outside [0, num_blocks) is not dereferenced: its keys are
+ *              left out and fa_sync_status reports FA_ERR_DEVICE.
+ * actual_seq_qlen, actual_seq_kvlen
+ *              host int64[B], cumulative as in fa_fwd: query rows per
+ *              sequence and cached keys per sequence (the handle's Skv =
+ *              the last kvlen entry).
+ * prefix       host int64[B] for modes 5/6, else ignored.
+ * Visibility: the handle's sparseMode row intervals per sequence (modes 0
+ * without a mask, 2..8), exactly as fa_fwd applies them to TND.
+ * Constraints (FA_ERR_* before any device work): a TND handle with no mask
+ * kind and sparse_mode != 1; 1 <= block_size <= 2^20; num_blocks >= 1;
+ * ceil(Skv_b / block_size) <= max_blocks for every b.
+ * The work is split over the keys (units of one sequence, one head, up to 4
+ * query rows and one chunk of keys) and each row's chunks are merged in a
+ * fixed order, so results are bitwise deterministic. Asynchronous, on
+ * cuda_stream; the handle's workspace holds the work list and the partial
+ * results.
+ */
+fa_status_t fa_fwd_paged(fa_handle_t h, const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* block_table, int64_t num_blocks, int32_t block_size,
+                         int32_t max_blocks, const int64_t* prefix, const int64_t* actual_seq_qlen,
+                         const int64_t* actual_seq_kvlen, void* o, float* lse, void* cuda_stream);
+
+/*
  * fa_mask_occupancy — the dense-mask pre-pass that fa_fwd and
  * fa_fwd_noalloc run before the attention kernel in sparseMode 1 (allMask)
  * and in sparseMode 0 with an attenMask ("sparseMode参数说明" page,

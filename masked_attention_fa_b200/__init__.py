@@ -101,6 +101,9 @@ def load_library():
     lib.fa_plan_stats.restype = st
     lib.fa_fwd_noalloc.argtypes = [dp, P, P, P, P, i64p, i64p, i64p, P, P, P]
     lib.fa_fwd_noalloc.restype = st
+    lib.fa_fwd_paged.argtypes = [P, P, P, P, P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                 i64p, i64p, i64p, P, P, P]
+    lib.fa_fwd_paged.restype = st
     lib.fa_mask_occupancy.argtypes = [dp, P, P, P, P]
     lib.fa_mask_occupancy.restype = st
     lib.fa_fwd_with_ranges.argtypes = [P, P, P, P, P, P, P, P, P]
@@ -114,7 +117,7 @@ def load_library():
 
 EXPORTED = ("fa_create", "fa_fwd", "fa_sync_status", "fa_destroy", "fa_last_error",
             "fa_version", "fa_validate", "fa_visible_pairs", "fa_tile_class", "fa_plan_stats",
-            "fa_fwd_noalloc", "fa_split_queries", "fa_mask_occupancy", "fa_fwd_with_ranges")
+            "fa_fwd_noalloc", "fa_split_queries", "fa_mask_occupancy", "fa_fwd_with_ranges", "fa_fwd_paged")
 
 
 def _check(status):
@@ -265,6 +268,19 @@ def fa_fwd_with_ranges(h, q, k, v, o, lse, atten_mask, ranges, stream=None):
                                              ctypes.c_void_p(_stream_int(stream, q.device))))
 
 
+def fa_fwd_paged(h, q, k_cache, v_cache, block_table, o, lse, actual_seq_qlen,
+                 actual_seq_kvlen, prefix=None, stream=None):
+    """Forward of a TND handle reading K/V from paged caches
+    [num_blocks, block_size, N, D] through block_table [B, max_blocks] (int32)."""
+    a = _Arrays(prefix, actual_seq_qlen, actual_seq_kvlen)
+    num_blocks, block_size = int(k_cache.shape[0]), int(k_cache.shape[1])
+    max_blocks = int(block_table.shape[1])
+    _check(load_library().fa_fwd_paged(h, _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                       _ptr(block_table), num_blocks, block_size, max_blocks,
+                                       *a.ptrs(), _ptr(o), _ptr(lse),
+                                       ctypes.c_void_p(_stream_int(stream, q.device))))
+
+
 def fa_fwd_noalloc(desc, q, k, v, o, lse, atten_mask=None, prefix=None, actual_seq_qlen=None,
                    actual_seq_kvlen=None, stream=None):
     """The allocation-free forward: no handle, the work list lives in the
@@ -344,6 +360,32 @@ class MaskedAttention:
         else:
             fa_fwd(self.handle, q, k, v, out, lse, atten_mask, prefix, actual_seq_qlen,
                    actual_seq_kvlen, stream)
+        return out, lse
+
+    def paged(self, q, k_cache, v_cache, block_table, actual_seq_qlen, actual_seq_kvlen,
+              prefix=None, out=None, lse=None, stream=None):
+        """O, lse of a TND handle with K/V in paged caches (see fa_fwd_paged)."""
+        import torch
+        oshape, lshape = self.out_shapes()
+        if out is None:
+            out = torch.empty(oshape, dtype=torch.bfloat16, device=q.device)
+        if lse is None:
+            lse = torch.empty(lshape, dtype=torch.float32, device=q.device)
+        for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("out", out)):
+            if t.dtype != torch.bfloat16 or not t.is_contiguous() or not t.is_cuda:
+                raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+        if block_table.dtype != torch.int32 or not block_table.is_contiguous():
+            raise ValueError("block_table must be a contiguous int32 tensor")
+        d = self.desc
+        if (k_cache.dim() != 4 or tuple(v_cache.shape) != tuple(k_cache.shape)
+                or k_cache.shape[2] != d.N or k_cache.shape[3] != d.D):
+            raise ValueError("k_cache and v_cache must both be [num_blocks, block_size, N, D]")
+        if block_table.dim() != 2 or block_table.shape[0] != d.B:
+            raise ValueError("block_table must be [B, max_blocks]")
+        if tuple(q.shape) != tuple(oshape):
+            raise ValueError(f"q must be {tuple(oshape)}")
+        fa_fwd_paged(self.handle, q, k_cache, v_cache, block_table, out, lse, actual_seq_qlen,
+                     actual_seq_kvlen, prefix, stream)
         return out, lse
 
     def occupancy(self, atten_mask, stream=None):

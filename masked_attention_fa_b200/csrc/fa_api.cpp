@@ -29,6 +29,10 @@ struct fa_handle_s {
   int32_t n_items = 0;
   int32_t n_seqs = 0;
   SeqRec geo0{};  // geometry of sequence 0 (every sequence's, outside TND)
+  // paged K/V calls: [header][SeqRec x B][PagedGroup x n_groups][PagedUnit x
+  // n_units] then the units' partial results (the plan key starts with -2)
+  int32_t n_groups = 0;
+  int64_t n_units = 0;
   // device workspace: [error word | pad to 256 B][SeqRec x B][WorkItem x n]
   // then, for a dense attenMask, the occupancy pre-pass's ranges and classes
   void* d_ws = nullptr;
@@ -416,6 +420,108 @@ fa_status_t fa_fwd_with_ranges(fa_handle_t h, const void* q, const void* k, cons
   return forward(h, q, k, v, atten_mask, ranges, nullptr, nullptr, nullptr, o, lse, cuda_stream);
 }
 
+fa_status_t fa_fwd_paged(fa_handle_t h, const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* block_table, int64_t num_blocks, int32_t block_size,
+                         int32_t max_blocks, const int64_t* prefix, const int64_t* actual_seq_qlen,
+                         const int64_t* actual_seq_kvlen, void* o, float* lse,
+                         void* cuda_stream) {
+  clear_error();
+  if (!h) return fail(FA_ERR_NULLPTR, "handle is NULL");
+  if (!q || !k_cache || !v_cache || !block_table || !o || !lse)
+    return fail(FA_ERR_NULLPTR, "q, k_cache, v_cache, block_table, o and lse are required");
+  const fa_desc_t* d = &h->desc;
+  fa_status_t st = validate_paged(d, prefix, actual_seq_qlen, actual_seq_kvlen, num_blocks,
+                                  block_size, max_blocks);
+  if (st != FA_OK) return st;
+  const uintptr_t align = (uintptr_t)q | (uintptr_t)k_cache | (uintptr_t)v_cache | (uintptr_t)o;
+  if (align & 15u)
+    return fail(FA_ERR_PARAM_INVALID, "q, k_cache, v_cache and o must be 16-byte aligned");
+  if (((uintptr_t)lse | (uintptr_t)block_table) & 3u)
+    return fail(FA_ERR_PARAM_INVALID, "lse and block_table must be 4-byte aligned");
+  st = bind_device(h);
+  if (st != FA_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  const int64_t D = d->D;
+  std::vector<int64_t> key = {-2, block_size, max_blocks};
+  key.insert(key.end(), actual_seq_qlen, actual_seq_qlen + d->B);
+  key.insert(key.end(), actual_seq_kvlen, actual_seq_kvlen + d->B);
+  if (d->sparse_mode == 5 || d->sparse_mode == 6) key.insert(key.end(), prefix, prefix + d->B);
+  const size_t part_unit = (size_t)kPagedRows * (size_t)(D + 2) * sizeof(float);
+  if (!h->plan_valid || key != h->plan_key) {
+    std::vector<SeqRec> recs = decode_geometry(d, prefix, actual_seq_qlen, actual_seq_kvlen, 0);
+    std::vector<PagedGroup> groups;
+    std::vector<PagedUnit> units;
+    build_paged(d, recs, 8 * (int64_t)h->num_sms, &groups, &units);
+    if (units.size() > (size_t)0x7fffffff || groups.size() > (size_t)0x7fffffff)
+      return fail(FA_ERR_UNSUPPORTED, "too many paged work units");
+    const size_t seq_bytes = align_up(recs.size() * sizeof(SeqRec), 256);
+    const size_t group_bytes = align_up(groups.size() * sizeof(PagedGroup), 256);
+    const size_t payload = seq_bytes + group_bytes + units.size() * sizeof(PagedUnit);
+    st = ensure_workspace(h, align_up(kHeaderBytes + payload, 256) + units.size() * part_unit);
+    if (st != FA_OK) return st;
+    st = ensure_stage(h, payload);
+    if (st != FA_OK) return st;
+    cudaError_t e = cudaEventSynchronize(h->stage_done);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+    if (h->any_call) {
+      e = cudaStreamWaitEvent(stream, h->last_call, 0);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+    }
+    uint8_t* hs = static_cast<uint8_t*>(h->h_stage);
+    std::memcpy(hs, recs.data(), recs.size() * sizeof(SeqRec));
+    if (!groups.empty()) std::memcpy(hs + seq_bytes, groups.data(), groups.size() * sizeof(PagedGroup));
+    if (!units.empty())
+      std::memcpy(hs + seq_bytes + group_bytes, units.data(), units.size() * sizeof(PagedUnit));
+    e = cudaMemcpyAsync(static_cast<uint8_t*>(h->d_ws) + kHeaderBytes, hs, payload,
+                        cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(paged work list)");
+    e = cudaEventRecord(h->stage_done, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    h->plan_key.swap(key);
+    h->plan_valid = true;
+    h->n_seqs = (int32_t)recs.size();
+    h->n_groups = (int32_t)groups.size();
+    h->n_units = (int64_t)units.size();
+    h->n_items = 0;
+  } else if (h->any_call) {
+    // The partial buffer is rewritten: order after the handle's last call.
+    cudaError_t e = cudaStreamWaitEvent(stream, h->last_call, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+  }
+  if (h->n_groups == 0) return FA_OK;  // no query rows
+  uint8_t* ws = static_cast<uint8_t*>(h->d_ws);
+  const size_t seq_bytes = align_up((size_t)h->n_seqs * sizeof(SeqRec), 256);
+  const size_t group_bytes = align_up((size_t)h->n_groups * sizeof(PagedGroup), 256);
+  const size_t payload = seq_bytes + group_bytes + (size_t)h->n_units * sizeof(PagedUnit);
+  PagedParams pp;
+  std::memset(&pp, 0, sizeof(pp));
+  pp.q = q;
+  pp.k_cache = k_cache;
+  pp.v_cache = v_cache;
+  pp.block_table = block_table;
+  pp.seqs = reinterpret_cast<const SeqRec*>(ws + kHeaderBytes);
+  pp.groups = reinterpret_cast<const PagedGroup*>(ws + kHeaderBytes + seq_bytes);
+  pp.units = reinterpret_cast<const PagedUnit*>(ws + kHeaderBytes + seq_bytes + group_bytes);
+  pp.part = reinterpret_cast<float*>(ws + align_up(kHeaderBytes + payload, 256));
+  pp.o = o;
+  pp.lse = lse;
+  pp.err_word = reinterpret_cast<unsigned int*>(ws);
+  pp.num_blocks = num_blocks;
+  pp.t_q = d->Sq;
+  pp.n_units = h->n_units;
+  pp.n_heads = (int32_t)d->N;
+  pp.block_size = block_size;
+  pp.max_blocks = max_blocks;
+  pp.n_groups = h->n_groups;
+  pp.scale_log2 = (float)(d->scale * 1.4426950408889634073599);
+  cudaError_t e = launch_paged((int)D, pp, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "paged kernel launch");
+  e = cudaEventRecord(h->last_call, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  h->any_call = true;
+  return FA_OK;
+}
+
 fa_status_t fa_mask_occupancy(const fa_desc_t* desc, const uint8_t* atten_mask,
                               uint8_t* tile_class, int32_t* ranges, void* cuda_stream) {
   clear_error();
@@ -466,6 +572,9 @@ fa_status_t fa_sync_status(fa_handle_t h) {
   if (word & kErrTimeout)
     return fail(FA_ERR_TIMEOUT, "a device-side wait gave up (site %u); outputs are undefined",
                 (word >> kErrWhereShift) & 0xffu);
+  if (word & kErrBadBlock)
+    return fail(FA_ERR_DEVICE,
+                "a block_table entry was outside [0, num_blocks); its keys were left out");
   return fail(FA_ERR_DEVICE, "device error word 0x%08x", word);
 }
 

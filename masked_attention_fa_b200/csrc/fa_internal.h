@@ -50,6 +50,24 @@ struct WorkItem {
 };
 static_assert(sizeof(WorkItem) == 16, "WorkItem layout");
 
+// Paged K/V forward (decode-shaped calls): a group is (sequence, head, up
+// to kPagedRows query rows); its visible keys are cut into units (chunks)
+// that run in parallel and are merged in order.
+constexpr int kPagedRows = 4;
+
+struct PagedGroup {
+  int32_t b, h;          // sequence, head
+  int32_t row0, nrows;   // query rows [row0, row0 + nrows) of the sequence
+  int32_t unit0, nunits; // its units, consecutive in the unit list
+};
+static_assert(sizeof(PagedGroup) == 24, "PagedGroup layout");
+
+struct PagedUnit {
+  int32_t group;
+  int32_t key0, key1;    // keys [key0, key1) of the sequence
+};
+static_assert(sizeof(PagedUnit) == 12, "PagedUnit layout");
+
 // KV tiles of one 128-row query sub-tile: [lo, hi) holds every tile with a
 // visible key; tiles in [full_lo, full_hi) need no element mask.
 struct TileRange {

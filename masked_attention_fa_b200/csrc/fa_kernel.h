@@ -88,6 +88,35 @@ struct SchedParams {
 constexpr int64_t kSortMaxItems = 65536;  // 2 bytes each in shared memory
 cudaError_t launch_schedule(const SchedParams& s, cudaStream_t stream);
 
+// ---------------------------------------------------------------- paged K/V
+// Decode-shaped forward over paged caches [num_blocks, block_size, N, D]:
+// work is split into groups (sequence, head, up to kPagedRows query rows)
+// and each group's visible keys into units (chunks) that run in parallel;
+// a merge pass combines each group's units in order.
+enum : uint32_t { kErrBadBlock = 1u << 16 };  // a block_table entry outside [0, num_blocks)
+
+struct PagedParams {
+  const void* q;               // bf16 [T_q, N, D]
+  const void* k_cache;         // bf16 [num_blocks, block_size, N, D]
+  const void* v_cache;
+  const int32_t* block_table;  // [B, max_blocks]
+  const SeqRec* seqs;
+  const PagedGroup* groups;
+  const PagedUnit* units;
+  float* part;                 // [n_units, kPagedRows, D + 2]: o, then m (log2 units), l
+  void* o;                     // bf16 [T_q, N, D]
+  float* lse;                  // [N, T_q]
+  unsigned int* err_word;
+  int64_t num_blocks;
+  int64_t t_q;
+  int64_t n_units;
+  int32_t n_heads, block_size, max_blocks, n_groups;
+  float scale_log2;
+};
+
+// Enqueue the partial and merge kernels for head dim D (64 or 128).
+cudaError_t launch_paged(int D, const PagedParams& p, cudaStream_t stream);
+
 // Build a 4-D bf16 tensor map over (D, S, N, B) with the given element
 // strides of S, N and B, boxes of 64 x 128 x 1 x 1, 128-byte swizzle.
 bool encode_operand_map(CUtensorMap* tm, const void* base, int64_t D, int64_t S, int64_t N,

@@ -273,6 +273,79 @@ std::vector<WorkItem> build_items(const fa_desc_t* d, const std::vector<SeqRec>&
   return items;
 }
 
+fa_status_t validate_paged(const fa_desc_t* d, const int64_t* prefix, const int64_t* cu_q,
+                           const int64_t* cu_kv, int64_t num_blocks, int32_t block_size,
+                           int32_t max_blocks) {
+  fa_status_t st = validate_call(d, prefix, cu_q, cu_kv, 0);
+  if (st != FA_OK) return st;
+  if (d->layout != FA_TND)
+    return fail(FA_ERR_UNSUPPORTED, "paged K/V needs a TND handle (packed query tokens)");
+  if (d->sparse_mode == 1 || d->mask_kind != FA_MASK_NONE)
+    return fail(FA_ERR_UNSUPPORTED, "paged K/V reads no attenMask (dense-mask modes need BNSD/BSND)");
+  if (block_size < 1 || block_size > (1 << 20))
+    return fail(FA_ERR_PARAM_INVALID, "block_size %d outside [1, 2^20]", block_size);
+  if (max_blocks < 1) return fail(FA_ERR_PARAM_INVALID, "max_blocks %d < 1", max_blocks);
+  if (num_blocks < 1) return fail(FA_ERR_PARAM_INVALID, "num_blocks %lld < 1", (long long)num_blocks);
+  if (num_blocks > (int64_t(1) << 40) / block_size)
+    return fail(FA_ERR_PARAM_INVALID, "num_blocks * block_size beyond 2^40 tokens");
+  for (int64_t b = 0; b < d->B; ++b) {
+    const int64_t skv = cu_kv[b] - (b ? cu_kv[b - 1] : 0);
+    if ((skv + block_size - 1) / block_size > max_blocks)
+      return fail(FA_ERR_SHAPE, "sequence %lld has %lld keys: more than max_blocks (%d) blocks of %d",
+                  (long long)b, (long long)skv, max_blocks, block_size);
+  }
+  return FA_OK;
+}
+
+// Groups in (sequence, head, row block) order, each with the chunks of its
+// visible key range [lo(first row), hi(last row)] (the row intervals are
+// monotone). The chunk length makes about target_units units in all,
+// between 256 and 16384 keys, a multiple of 64.
+void build_paged(const fa_desc_t* d, const std::vector<SeqRec>& recs, int64_t target_units,
+                 std::vector<PagedGroup>* groups, std::vector<PagedUnit>* units) {
+  groups->clear();
+  units->clear();
+  struct Span { int64_t lo, hi; };
+  std::vector<Span> spans;
+  int64_t total = 0;
+  for (const SeqRec& s : recs) {
+    for (int64_t r0 = 0; r0 < s.sq; r0 += kPagedRows) {
+      const int64_t r1 = imin64(r0 + kPagedRows, s.sq) - 1;
+      const int64_t lo = imax64(0, row_lo(s, r0));
+      const int64_t hi = imin64(int64_t(s.skv) - 1, row_hi(s, r1));
+      spans.push_back(Span{lo, hi});
+      if (hi >= lo) total += (hi - lo + 1) * d->N;
+    }
+  }
+  int64_t chunk = target_units > 0 ? (total + target_units - 1) / target_units : 256;
+  chunk = imin64(imax64(chunk, 256), 16384);
+  chunk = (chunk + 63) / 64 * 64;
+  size_t si = 0;
+  for (size_t b = 0; b < recs.size(); ++b) {
+    const SeqRec& s = recs[b];
+    const size_t first = si;
+    for (int64_t h = 0; h < d->N; ++h) {
+      si = first;
+      for (int64_t r0 = 0; r0 < s.sq; r0 += kPagedRows, ++si) {
+        const Span sp = spans[si];
+        PagedGroup g;
+        g.b = (int32_t)b;
+        g.h = (int32_t)h;
+        g.row0 = (int32_t)r0;
+        g.nrows = (int32_t)(imin64(r0 + kPagedRows, s.sq) - r0);
+        g.unit0 = (int32_t)units->size();
+        g.nunits = 0;
+        for (int64_t k0 = sp.lo; k0 <= sp.hi; k0 += chunk) {
+          units->push_back(PagedUnit{(int32_t)groups->size(), (int32_t)k0,
+                                     (int32_t)imin64(k0 + chunk, sp.hi + 1)});
+          ++g.nunits;
+        }
+        groups->push_back(g);
+      }
+    }
+  }
+}
+
 int64_t visible_pairs(const fa_desc_t* d, const std::vector<SeqRec>& recs) {
   int64_t total = 0;
   for (const SeqRec& s : recs) {
