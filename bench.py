@@ -187,7 +187,52 @@ def prepass_bytes(w):
     return planes * (per_plane + 2 * n_qt * n_kt + 16 * n_qt)
 
 
+def paged_bytes(w):
+    """Algorithmic bytes of a paged forward: every visible cached key and
+    value row once per head (bf16), q and O (bf16) and lse (fp32). Each
+    sequence's visible keys run from its first row's lowest to its last
+    row's highest key; the paged workloads are rightDownCausal, whose last
+    row sees every key."""
+    assert w.sparse_mode == 3
+    keys = sum(skv for _, skv in w.seq_lens())
+    return 2 * keys * w.N * w.D * 2 + 2 * w.Sq * w.N * w.D * 2 + w.N * w.Sq * 4
+
+
+def cpu_baseline_sample_paged(w, inputs, seconds):
+    """The paged oracle on (sequence, head 0) problems, sequences in turn,
+    each with its blocks of head 0 gathered to the host once."""
+    import numpy as np
+    import oracle
+    from oracle import Problem
+    lens = w.seq_lens()
+    table = inputs["block_table"].cpu()
+    cases = []
+    for bi, (sq, skv) in enumerate(lens):
+        nblk = -(-skv // w.block_size)
+        blocks = table[bi, :nblk].long().to(inputs["k_cache"].device)
+        q0 = int(w.actual_seq_qlen[bi - 1]) if bi else 0
+        cases.append((sq, skv, nblk, inputs["q"][q0:q0 + sq, :1].cpu(),
+                      inputs["k_cache"][blocks][:, :, :1].cpu(),
+                      inputs["v_cache"][blocks][:, :, :1].cpu()))
+    pairs, elapsed, done = 0, 0.0, 0
+    while elapsed < seconds and done < 100000:
+        sq, skv, nblk, q, kc, vc = cases[done % len(cases)]
+        pb = Problem("TND", 1, 1, sq, skv, w.D, sparse_mode=w.sparse_mode, scale=w.scale,
+                     actual_seq_qlen=[sq], actual_seq_kvlen=[skv])
+        t0 = time.perf_counter()
+        oracle.attention_paged(pb, q, kc, vc, np.arange(nblk, dtype=np.int32)[None], w.block_size)
+        elapsed += time.perf_counter() - t0
+        pairs += sq * skv
+        done += 1
+    tflops = 4.0 * w.D * pairs / elapsed / 1e12
+    desc = (f"{done} (sequence, head 0) problems of {w.name}, sequences in turn, K/V blocks "
+            f"gathered to the host; {pairs} visible pairs in {elapsed:.1f} s")
+    return tflops, oracle.num_threads(), desc
+
+
 def cpu_baseline_sample(w, inputs, seconds):
+    if w.block_size is not None:
+        return cpu_baseline_sample_paged(w, inputs, seconds)
     """Time the oracle (as it stands) on a bounded sample of query rows of the
     same workload; returns (TFLOP/s, cores, description)."""
     import numpy as np
@@ -244,7 +289,12 @@ def run_reference(args):
     from masked_attention_fa_b200.workloads import named_workloads, make_inputs
     import oracle
     w = named_workloads()[args.workload]
-    inputs = make_inputs(w)
+    if w.block_size is not None:
+        # gigabytes of cache values: drawn by the GPU when there is one
+        import torch
+        inputs = make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
+    else:
+        inputs = make_inputs(w)
     per_step = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
     vals = []
     desc = None
@@ -288,8 +338,13 @@ def main():
     dev = torch.device("cuda", local)
 
     w = named_workloads()[args.workload]
-    inputs = make_inputs(w)
-    q, k, v = (inputs[x].to(dev) for x in ("q", "k", "v"))
+    paged = w.block_size is not None
+    if paged:  # caches drawn on the device (gigabytes; see workloads.paged_inputs)
+        inputs = make_inputs(w, device=dev)
+        q, kc, vc, table = (inputs[x] for x in ("q", "k_cache", "v_cache", "block_table"))
+    else:
+        inputs = make_inputs(w)
+        q, k, v = (inputs[x].to(dev) for x in ("q", "k", "v"))
     mask = inputs["mask"].to(dev) if inputs["mask"] is not None else None
     arrays = workload_args(w)
     attn = fa.MaskedAttention(w.layout, w.B, w.N, w.Sq, w.Skv, w.D, w.sparse_mode, w.pre_tokens,
@@ -315,7 +370,10 @@ def main():
         fa.fa_mask_occupancy(attn.desc, mask, tile_class=tile_cls, ranges=ranges, stream=stream)
 
     def attention():
-        if dense:
+        if paged:
+            attn.paged(q, kc, vc, table, w.actual_seq_qlen, w.actual_seq_kvlen, out=o, lse=lse,
+                       stream=stream)
+        elif dense:
             attn(q, k, v, atten_mask=mask, out=o, lse=lse, stream=stream, ranges=ranges)
         else:
             attn(q, k, v, atten_mask=mask, out=o, lse=lse, stream=stream, **arrays)
@@ -373,7 +431,10 @@ def main():
     # directions at once). Events order the reuse of each buffer pair.
     e2e = None
     if not args.no_e2e:
-        host_in = [inputs[x].pin_memory() for x in ("q", "k", "v")]
+        if paged:  # the caches are the state: resident; q and the block table go up
+            host_in = [inputs["q"].cpu().pin_memory(), inputs["block_table"].cpu().pin_memory()]
+        else:
+            host_in = [inputs[x].pin_memory() for x in ("q", "k", "v")]
         if dense:
             host_in.append(inputs["mask"].pin_memory())
         dev_in = [[torch.empty_like(x, device=dev) for x in host_in] for _ in range(2)]
@@ -398,9 +459,14 @@ def main():
             stream.wait_event(ev_up[b])
             if used[b]:
                 stream.wait_event(ev_down[b])  # step i-2's outputs have left the device
-            qb, kb, vb = dev_in[b][:3]
-            mb = dev_in[b][3] if dense else None
-            attn(qb, kb, vb, atten_mask=mb, out=dev_o[b], lse=dev_l[b], stream=stream, **arrays)
+            if paged:
+                attn.paged(dev_in[b][0], kc, vc, dev_in[b][1], w.actual_seq_qlen,
+                           w.actual_seq_kvlen, out=dev_o[b], lse=dev_l[b], stream=stream)
+            else:
+                qb, kb, vb = dev_in[b][:3]
+                mb = dev_in[b][3] if dense else None
+                attn(qb, kb, vb, atten_mask=mb, out=dev_o[b], lse=dev_l[b], stream=stream,
+                     **arrays)
             ev_fwd[b].record(stream)
             with torch.cuda.stream(down):
                 down.wait_event(ev_fwd[b])
@@ -445,6 +511,17 @@ def main():
                     "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
                     "kernel": f"fa_fwd_sm100<{w.D}, {'true' if dense else 'false'}>",
                     "kernel_ms": kern_ms}
+        if paged:
+            # A few query rows per sequence: every cached K/V byte is used for a
+            # handful of FMAs, so HBM bounds the path, not the tensor cores.
+            nbytes = paged_bytes(w)
+            gbs = nbytes / (kern_ms * 1e-3) / 1e9
+            hbm = float(peaks["hbm_gbs"])
+            roofline = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                        "frac": gbs / hbm, "traffic": traffic, "bytes_per_launch": nbytes,
+                        "peak_source": f"{peak_src} hbm_gbs",
+                        "kernel": f"paged_partial<{w.D}> + paged_merge<{w.D}>",
+                        "kernel_ms": kern_ms, "tflops": achieved}
         if dense:
             roofline["kernel_ms_includes"] = ("the one-block work-list rebuild "
                                               "(occupancy_schedule) launched just before it")
@@ -470,10 +547,13 @@ def main():
                            "Sq": w.Sq, "Skv": w.Skv, "D": w.D, "sparse_mode": w.sparse_mode,
                            "visible_pairs": pairs, "per_rank": "independent copy",
                            "l2": "256 MiB buffer written between timed steps (cold L2)",
+                           **({"block_size": w.block_size, "kv_cache": "paged, resident"}
+                              if paged else {}),
                            "parallelism": f"replicas x{world}"},
                 "frac_of_peak": value / world / peak,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": args.steps * (4 if dense else 1), "clocks": clocks,
+                "gpu_launches": args.steps * (4 if dense else (2 if paged else 1)),
+                "clocks": clocks,
                 "ms_min": min(times_ms), "ms_median": statistics.median(times_ms)}
         if prepass_line is not None:
             line["prepass"] = prepass_line

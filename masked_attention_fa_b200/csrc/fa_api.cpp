@@ -7,6 +7,7 @@
 // persistent kernel on the caller's stream.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -33,6 +34,7 @@ struct fa_handle_s {
   // n_units] then the units' partial results (the plan key starts with -2)
   int32_t n_groups = 0;
   int64_t n_units = 0;
+  int32_t paged_rows = 0;  // most query rows in one group
   // device workspace: [error word | pad to 256 B][SeqRec x B][WorkItem x n]
   // then, for a dense attenMask, the occupancy pre-pass's ranges and classes
   void* d_ws = nullptr;
@@ -446,12 +448,15 @@ fa_status_t fa_fwd_paged(fa_handle_t h, const void* q, const void* k_cache, cons
   key.insert(key.end(), actual_seq_qlen, actual_seq_qlen + d->B);
   key.insert(key.end(), actual_seq_kvlen, actual_seq_kvlen + d->B);
   if (d->sparse_mode == 5 || d->sparse_mode == 6) key.insert(key.end(), prefix, prefix + d->B);
-  const size_t part_unit = (size_t)kPagedRows * (size_t)(D + 2) * sizeof(float);
+  const int32_t hpu = paged_heads_per_unit(d->N, (int)D);
+  const size_t part_unit = (size_t)hpu * kPagedRows * (size_t)(D + 4) * sizeof(float);
   if (!h->plan_valid || key != h->plan_key) {
     std::vector<SeqRec> recs = decode_geometry(d, prefix, actual_seq_qlen, actual_seq_kvlen, 0);
     std::vector<PagedGroup> groups;
     std::vector<PagedUnit> units;
-    build_paged(d, recs, 8 * (int64_t)h->num_sms, &groups, &units);
+    int32_t max_rows = 0;
+    for (const SeqRec& r : recs) max_rows = std::max(max_rows, std::min(r.sq, (int32_t)kPagedRows));
+    build_paged(d, recs, paged_slots((int)D, max_rows, hpu, h->num_sms), hpu, &groups, &units);
     if (units.size() > (size_t)0x7fffffff || groups.size() > (size_t)0x7fffffff)
       return fail(FA_ERR_UNSUPPORTED, "too many paged work units");
     const size_t seq_bytes = align_up(recs.size() * sizeof(SeqRec), 256);
@@ -483,6 +488,8 @@ fa_status_t fa_fwd_paged(fa_handle_t h, const void* q, const void* k_cache, cons
     h->n_groups = (int32_t)groups.size();
     h->n_units = (int64_t)units.size();
     h->n_items = 0;
+    h->paged_rows = 0;
+    for (const PagedGroup& g : groups) h->paged_rows = std::max(h->paged_rows, g.nrows);
   } else if (h->any_call) {
     // The partial buffer is rewritten: order after the handle's last call.
     cudaError_t e = cudaStreamWaitEvent(stream, h->last_call, 0);
@@ -513,8 +520,9 @@ fa_status_t fa_fwd_paged(fa_handle_t h, const void* q, const void* k_cache, cons
   pp.block_size = block_size;
   pp.max_blocks = max_blocks;
   pp.n_groups = h->n_groups;
+  pp.heads_per_unit = hpu;
   pp.scale_log2 = (float)(d->scale * 1.4426950408889634073599);
-  cudaError_t e = launch_paged((int)D, pp, stream);
+  cudaError_t e = launch_paged((int)D, h->paged_rows, pp, stream);
   if (e != cudaSuccess) return cuda_fail(e, "paged kernel launch");
   e = cudaEventRecord(h->last_call, stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");

@@ -51,22 +51,28 @@ struct WorkItem {
 static_assert(sizeof(WorkItem) == 16, "WorkItem layout");
 
 // Paged K/V forward (decode-shaped calls): a group is (sequence, head, up
-// to kPagedRows query rows); its visible keys are cut into units (chunks)
-// that run in parallel and are merged in order.
+// to kPagedRows query rows); its visible keys are cut into chunks. A unit
+// is one chunk of one row block of one sequence for a run of heads (one CTA
+// reads whole token rows of the cache); its partial results are merged per
+// group in chunk order.
 constexpr int kPagedRows = 4;
 
 struct PagedGroup {
   int32_t b, h;          // sequence, head
   int32_t row0, nrows;   // query rows [row0, row0 + nrows) of the sequence
-  int32_t unit0, nunits; // its units, consecutive in the unit list
+  int32_t unit0, nunits; // its units: unit0 + c * ustride, c < nunits
+  int32_t ustride;       // units between consecutive chunks of the group
+  int32_t hslot;         // the head's slot in those units' partial results
 };
-static_assert(sizeof(PagedGroup) == 24, "PagedGroup layout");
+static_assert(sizeof(PagedGroup) == 32, "PagedGroup layout");
 
 struct PagedUnit {
-  int32_t group;
+  int32_t b;             // sequence
+  int32_t row0, nrows;   // query rows of the sequence
+  int32_t h0;            // first head (the unit covers heads h0 .. h0 + heads per unit - 1)
   int32_t key0, key1;    // keys [key0, key1) of the sequence
 };
-static_assert(sizeof(PagedUnit) == 12, "PagedUnit layout");
+static_assert(sizeof(PagedUnit) == 24, "PagedUnit layout");
 
 // KV tiles of one 128-row query sub-tile: [lo, hi) holds every tile with a
 // visible key; tiles in [full_lo, full_hi) need no element mask.

@@ -103,7 +103,7 @@ struct PagedParams {
   const SeqRec* seqs;
   const PagedGroup* groups;
   const PagedUnit* units;
-  float* part;                 // [n_units, kPagedRows, D + 2]: o, then m (log2 units), l
+  float* part;                 // per (unit, head, row): o[D], m (log2 units), l, 2 pad (D + 4 floats)
   void* o;                     // bf16 [T_q, N, D]
   float* lse;                  // [N, T_q]
   unsigned int* err_word;
@@ -111,11 +111,19 @@ struct PagedParams {
   int64_t t_q;
   int64_t n_units;
   int32_t n_heads, block_size, max_blocks, n_groups;
+  int32_t heads_per_unit;      // heads one unit (CTA) covers; part is [unit][head][row][D + 2]
   float scale_log2;
 };
 
-// Enqueue the partial and merge kernels for head dim D (64 or 128).
-cudaError_t launch_paged(int D, const PagedParams& p, cudaStream_t stream);
+// Heads one paged unit covers for N heads of dimension D: whole warps of
+// D / 16 threads per head, at most 256 threads.
+int paged_heads_per_unit(int64_t n_heads, int D);
+// CTAs of the partial kernel resident at once on num_sms SMs.
+int paged_slots(int D, int max_rows, int heads_per_unit, int num_sms);
+
+// Enqueue the partial and merge kernels for head dim D (64 or 128);
+// max_rows: the most query rows any group holds.
+cudaError_t launch_paged(int D, int max_rows, const PagedParams& p, cudaStream_t stream);
 
 // Build a 4-D bf16 tensor map over (D, S, N, B) with the given element
 // strides of S, N and B, boxes of 64 x 128 x 1 x 1, 128-byte swizzle.

@@ -14,14 +14,17 @@
 // bandwidth. It is split over the keys so that a few long sequences still
 // fill the GPU:
 //
-//   paged_partial  one CTA (4 warps) per (sequence, head, group of up to
-//                  kPagedRows query rows, chunk of keys). Lane l of a warp
-//                  owns D/32 consecutive dimensions of q, k, v and o; a warp
-//                  takes 8 keys per step with all their loads in flight, forms
-//                  each score with a butterfly sum over the warp and runs
-//                  the online softmax (running max m, running sum l) per row.
-//                  The four warps' (m, l, o) are combined in shared memory
-//                  and the chunk's partial is written in fp32.
+//   paged_partial  one CTA per (sequence, row block of up to kPagedRows
+//                  query rows, chunk of keys, run of up to 256 * 16 / D
+//                  heads). D / 16 threads share a head, each with 16
+//                  dimensions of q, k, v and o, so for every key the CTA reads
+//                  whole token rows of the cache (a token's heads are adjacent
+//                  in the layout) with 32-byte loads, several keys in flight.
+//                  A score is a sum over the head's threads (xor shuffles);
+//                  each (head, row) runs the online softmax (running max m,
+//                  running sum l) over the whole chunk and writes its partial
+//                  (o, m, l) in fp32. The unit's block ids are staged in
+//                  shared memory.
 //   paged_merge    one warp per (group, row) combines the chunks of its group
 //                  in chunk order (a fixed order, so the result is the same
 //                  on every run), divides by l and writes O (bf16) and lse.
@@ -36,35 +39,19 @@
 namespace fa {
 namespace {
 
-constexpr int kPagedWarps = 4;
-constexpr int kPagedKeys = 8;  // keys per warp step (loads in flight)
+constexpr int kSlice = 16;        // dimensions per thread
+constexpr int kPartPad = 4;       // a partial row: o[D], m, l, two pad floats (16-byte rows)
+constexpr int kTableStage = 512;  // block ids of a unit staged in shared memory
 constexpr float kLn2 = 0.69314718055994530942f;
 
-template <int D>
-struct PagedVec;
-template <>
-struct PagedVec<128> {  // 4 bf16 per lane
-  using T = uint2;
-  static __device__ __forceinline__ void unpack(const T& v, float (&f)[4]) {
-    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
-    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
-    const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
-    f[0] = fa.x, f[1] = fa.y, f[2] = fb.x, f[3] = fb.y;
-  }
-};
-template <>
-struct PagedVec<64> {  // 2 bf16 per lane
-  using T = uint32_t;
-  static __device__ __forceinline__ void unpack(const T& v, float (&f)[2]) {
-    const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v));
-    f[0] = fa.x, f[1] = fa.y;
-  }
-};
-
-__device__ __forceinline__ float warp_sum(float x) {
+__device__ __forceinline__ void unpack8(const uint4& v, float* f) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int d = 16; d >= 1; d >>= 1) x += __shfl_xor_sync(0xffffffffu, x, d);
-  return x;
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
 }
 
 // Rescale an accumulator to a larger running maximum (log2 units).
@@ -72,133 +59,141 @@ __device__ __forceinline__ float rescale(float m_old, float m_new) {
   return m_old == -INFINITY ? 0.f : exp2f(m_old - m_new);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kPagedWarps * 32) paged_partial(const PagedParams p) {
-  constexpr int V = D / 32;  // dimensions per lane
-  using Vec = PagedVec<D>;
-  using T = typename Vec::T;
-  __shared__ float sm_m[kPagedWarps][kPagedRows], sm_l[kPagedWarps][kPagedRows];
-  __shared__ float sm_o[kPagedWarps][kPagedRows][D];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// One CTA per unit: heads [h0, h0 + HC) of one row block of one sequence
+// over the keys [key0, key1). Thread t serves head h0 + t / L (L = D / 16
+// threads per head) and dimensions [16 (t % L), 16 (t % L) + 16), so for
+// every key the CTA reads whole token rows of the cache (all heads are
+// adjacent in the layout). R: rows a unit may hold (1 for decode calls);
+// KEYS: keys whose loads are in flight together.
+template <int D, int R, int KEYS>
+__global__ void __launch_bounds__(256) paged_partial(const PagedParams p) {
+  constexpr int L = D / kSlice;
+  __shared__ int32_t sm_blk[kTableStage];
   const PagedUnit u = p.units[blockIdx.x];
-  const PagedGroup g = p.groups[u.group];
-  const SeqRec sr = p.seqs[g.b];
-  // This lane's slice of q for the group's rows, pre-multiplied by scale * log2(e).
-  float q[kPagedRows][V];
-  int jlo[kPagedRows], jhi[kPagedRows];
+  const SeqRec sr = p.seqs[u.b];
+  const int hl = threadIdx.x / L, sl = threadIdx.x % L;
+  const int h = u.h0 + hl;
+  const bool live = h < p.n_heads;
+  const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(p.q);
+  float q[R][kSlice];
+  int jlo[R], jhi[R];
 #pragma unroll
-  for (int r = 0; r < kPagedRows; ++r) {
+  for (int r = 0; r < R; ++r) {
     jlo[r] = 1, jhi[r] = 0;
 #pragma unroll
-    for (int x = 0; x < V; ++x) q[r][x] = 0.f;
-    if (r < g.nrows) {
-      const int64_t i = (int64_t)g.row0 + r;  // row inside the sequence
+    for (int x = 0; x < kSlice; ++x) q[r][x] = 0.f;
+    if (r < u.nrows) {
+      const int64_t i = (int64_t)u.row0 + r;  // row inside the sequence
       jlo[r] = (int)imax64(0, row_lo(sr, i));
       jhi[r] = (int)imin64((int64_t)sr.skv - 1, row_hi(sr, i));
-      const T qv = *reinterpret_cast<const T*>(
-          reinterpret_cast<const __nv_bfloat16*>(p.q) +
-          (((int64_t)sr.q_off + i) * p.n_heads + g.h) * D + lane * V);
-      float f[V];
-      Vec::unpack(qv, f);
+      if (live) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            qb + (((int64_t)sr.q_off + i) * p.n_heads + h) * D + sl * kSlice);
+        unpack8(src[0], q[r]);
+        unpack8(src[1], q[r] + 8);
 #pragma unroll
-      for (int x = 0; x < V; ++x) q[r][x] = f[x] * p.scale_log2;
+        for (int x = 0; x < kSlice; ++x) q[r][x] *= p.scale_log2;
+      }
     }
   }
-  float m[kPagedRows], l[kPagedRows], o[kPagedRows][V];
+  float m[R], l[R], o[R][kSlice];
 #pragma unroll
-  for (int r = 0; r < kPagedRows; ++r) {
+  for (int r = 0; r < R; ++r) {
     m[r] = -INFINITY, l[r] = 0.f;
 #pragma unroll
-    for (int x = 0; x < V; ++x) o[r][x] = 0.f;
+    for (int x = 0; x < kSlice; ++x) o[r][x] = 0.f;
   }
   const __nv_bfloat16* kc = reinterpret_cast<const __nv_bfloat16*>(p.k_cache);
   const __nv_bfloat16* vc = reinterpret_cast<const __nv_bfloat16*>(p.v_cache);
-  const int32_t* table = p.block_table + (int64_t)g.b * p.max_blocks;
+  const int32_t* table = p.block_table + (int64_t)u.b * p.max_blocks;
+  // The unit's block ids, read once into shared memory (units hold keys, so
+  // key1 > key0 and the blocks are table entries [blk0, blk0 + nblk)).
+  const int blk0 = u.key0 / p.block_size;
+  const int nblk = (u.key1 - 1) / p.block_size - blk0 + 1;
+  const bool staged = nblk <= kTableStage;
+  if (staged)
+    for (int t = threadIdx.x; t < nblk; t += blockDim.x) sm_blk[t] = __ldg(table + blk0 + t);
+  __syncthreads();
   bool bad = false;
-  // Keys [key0, key1): warp w takes steps of kPagedKeys keys, round robin.
-  for (int j0 = u.key0 + warp * kPagedKeys; j0 < u.key1; j0 += kPagedWarps * kPagedKeys) {
-    T kv[kPagedKeys], vv[kPagedKeys];
-    bool ok[kPagedKeys];
+  for (int j0 = u.key0; j0 < u.key1; j0 += KEYS) {
+    uint4 kv[KEYS][2], vv[KEYS][2];
+    bool ok[KEYS];
 #pragma unroll
-    for (int e = 0; e < kPagedKeys; ++e) {
+    for (int e = 0; e < KEYS; ++e) {
       const int j = j0 + e;
       ok[e] = false;
       if (j < u.key1) {
-        const int32_t blk = __ldg(table + j / p.block_size);
+        const int32_t blk =
+            staged ? sm_blk[j / p.block_size - blk0] : __ldg(table + j / p.block_size);
         if (blk >= 0 && (int64_t)blk < p.num_blocks) {
-          const int64_t slot = (int64_t)blk * p.block_size + j % p.block_size;
-          const int64_t off = (slot * p.n_heads + g.h) * D + lane * V;
-          kv[e] = __ldg(reinterpret_cast<const T*>(kc + off));
-          vv[e] = __ldg(reinterpret_cast<const T*>(vc + off));
           ok[e] = true;
+          if (live) {
+            const int64_t slot = (int64_t)blk * p.block_size + j % p.block_size;
+            const int64_t off = (slot * p.n_heads + h) * D + sl * kSlice;
+            const uint4* ks = reinterpret_cast<const uint4*>(kc + off);
+            const uint4* vs = reinterpret_cast<const uint4*>(vc + off);
+            kv[e][0] = __ldg(ks);
+            kv[e][1] = __ldg(ks + 1);
+            vv[e][0] = __ldg(vs);
+            vv[e][1] = __ldg(vs + 1);
+          } else {
+            kv[e][0] = kv[e][1] = vv[e][0] = vv[e][1] = make_uint4(0u, 0u, 0u, 0u);
+          }
         } else {
           bad = true;
         }
       }
     }
 #pragma unroll
-    for (int e = 0; e < kPagedKeys; ++e) {
-      if (!ok[e]) continue;  // warp-uniform: every lane saw the same block id
+    for (int e = 0; e < KEYS; ++e) {
+      if (!ok[e]) continue;  // the same for every thread: one block id per key
       const int j = j0 + e;
-      float kf[V], vf[V];
-      Vec::unpack(kv[e], kf);
-      Vec::unpack(vv[e], vf);
+      float kf[kSlice], vf[kSlice];
+      unpack8(kv[e][0], kf);
+      unpack8(kv[e][1], kf + 8);
+      unpack8(vv[e][0], vf);
+      unpack8(vv[e][1], vf + 8);
 #pragma unroll
-      for (int r = 0; r < kPagedRows; ++r) {
-        if (r >= g.nrows) break;
-        float part = 0.f;
+      for (int r = 0; r < R; ++r) {
+        if (r >= u.nrows) break;
+        float s = 0.f;
 #pragma unroll
-        for (int x = 0; x < V; ++x) part = fmaf(q[r][x], kf[x], part);
-        const float s = warp_sum(part);
+        for (int x = 0; x < kSlice; ++x) s = fmaf(q[r][x], kf[x], s);
+#pragma unroll
+        for (int d = 1; d < L; d <<= 1) s += __shfl_xor_sync(0xffffffffu, s, d);
         if (j < jlo[r] || j > jhi[r]) continue;
         if (s > m[r]) {
           const float a = rescale(m[r], s);
           l[r] *= a;
 #pragma unroll
-          for (int x = 0; x < V; ++x) o[r][x] *= a;
+          for (int x = 0; x < kSlice; ++x) o[r][x] *= a;
           m[r] = s;
         }
         const float pj = exp2f(s - m[r]);
         l[r] += pj;
 #pragma unroll
-        for (int x = 0; x < V; ++x) o[r][x] = fmaf(pj, vf[x], o[r][x]);
+        for (int x = 0; x < kSlice; ++x) o[r][x] = fmaf(pj, vf[x], o[r][x]);
       }
     }
   }
-  if (bad && lane == 0) atomicOr(p.err_word, kErrBadBlock);
-  // Combine the four warps.
+  if (bad && threadIdx.x == 0) atomicOr(p.err_word, kErrBadBlock);
+  if (!live) return;
+  float* out = p.part + ((int64_t)blockIdx.x * p.heads_per_unit + hl) * kPagedRows * (D + kPartPad);
 #pragma unroll
-  for (int r = 0; r < kPagedRows; ++r) {
-    if (lane == 0) {
-      sm_m[warp][r] = m[r];
-      sm_l[warp][r] = l[r];
-    }
+  for (int r = 0; r < R; ++r) {
+    if (r >= u.nrows) break;
+    float4* dst = reinterpret_cast<float4*>(out + r * (D + kPartPad) + sl * kSlice);
 #pragma unroll
-    for (int x = 0; x < V; ++x) sm_o[warp][r][lane * V + x] = o[r][x];
-  }
-  __syncthreads();
-  // Thread t writes dimension (t % D) of rows t / D, t / D + 128 / D, ...
-  float* out = p.part + (int64_t)blockIdx.x * kPagedRows * (D + 2);
-  for (int idx = threadIdx.x; idx < kPagedRows * D; idx += kPagedWarps * 32) {
-    const int r = idx / D, x = idx % D;
-    float mm = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kPagedWarps; ++w) mm = fmaxf(mm, sm_m[w][r]);
-    float acc = 0.f, ll = 0.f;
-#pragma unroll
-    for (int w = 0; w < kPagedWarps; ++w) {
-      const float a = rescale(sm_m[w][r], mm);
-      acc += sm_o[w][r][x] * a;
-      ll += sm_l[w][r] * a;
-    }
-    out[r * (D + 2) + x] = acc;
-    if (x == 0) {
-      out[r * (D + 2) + D] = mm;
-      out[r * (D + 2) + D + 1] = ll;
+    for (int x = 0; x < kSlice / 4; ++x)
+      dst[x] = make_float4(o[r][4 * x], o[r][4 * x + 1], o[r][4 * x + 2], o[r][4 * x + 3]);
+    if (sl == 0) {
+      out[r * (D + kPartPad) + D] = m[r];
+      out[r * (D + kPartPad) + D + 1] = l[r];
     }
   }
 }
 
+// One warp per (group, row): the group's chunks in chunk order.
 template <int D>
 __global__ void __launch_bounds__(128) paged_merge(const PagedParams p) {
   const int lane = threadIdx.x & 31;
@@ -209,14 +204,17 @@ __global__ void __launch_bounds__(128) paged_merge(const PagedParams p) {
   if (r >= g.nrows) return;
   const SeqRec sr = p.seqs[g.b];
   const int64_t t = (int64_t)sr.q_off + g.row0 + r;  // query token
+  auto part_of = [&](int c) {
+    const int64_t unit = (int64_t)g.unit0 + (int64_t)c * g.ustride;
+    return p.part + ((unit * p.heads_per_unit + g.hslot) * kPagedRows + r) * (D + kPartPad);
+  };
   float mm = -INFINITY;
-  for (int c = 0; c < g.nunits; ++c)
-    mm = fmaxf(mm, p.part[((int64_t)(g.unit0 + c) * kPagedRows + r) * (D + 2) + D]);
+  for (int c = 0; c < g.nunits; ++c) mm = fmaxf(mm, part_of(c)[D]);
   float acc[D / 32], ll = 0.f;
 #pragma unroll
   for (int x = 0; x < D / 32; ++x) acc[x] = 0.f;
   for (int c = 0; c < g.nunits; ++c) {
-    const float* part = p.part + ((int64_t)(g.unit0 + c) * kPagedRows + r) * (D + 2);
+    const float* part = part_of(c);
     const float a = rescale(part[D], mm);
     ll += part[D + 1] * a;
 #pragma unroll
@@ -230,23 +228,53 @@ __global__ void __launch_bounds__(128) paged_merge(const PagedParams p) {
     p.lse[(int64_t)g.h * p.t_q + t] = ll > 0.f ? (mm + log2f(ll)) * kLn2 : -INFINITY;
 }
 
+template <int D>
+cudaError_t launch_d(int max_rows, const PagedParams& p, cudaStream_t stream) {
+  const int threads = p.heads_per_unit * (D / kSlice);
+  const int units = (int)p.n_units;
+  if (units > 0) {
+    if (max_rows <= 1) paged_partial<D, 1, 4><<<units, threads, 0, stream>>>(p);
+    else paged_partial<D, kPagedRows, 2><<<units, threads, 0, stream>>>(p);
+  }
+  const int64_t merge_blocks = ((int64_t)p.n_groups * kPagedRows + 3) / 4;
+  if (merge_blocks > 0) paged_merge<D><<<(int)merge_blocks, 128, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
-cudaError_t launch_paged(int D, const PagedParams& p, cudaStream_t stream) {
-  if (p.n_units <= 0 && p.n_groups <= 0) return cudaSuccess;
-  const int64_t merge_warps = (int64_t)p.n_groups * kPagedRows;
-  const int64_t merge_blocks = (merge_warps + 3) / 4;
-  if (p.n_units > 0x7fffffff || merge_blocks > 0x7fffffff) return cudaErrorInvalidValue;
-  if (D == 128) {
-    if (p.n_units > 0) paged_partial<128><<<(int)p.n_units, kPagedWarps * 32, 0, stream>>>(p);
-    if (merge_blocks > 0) paged_merge<128><<<(int)merge_blocks, 128, 0, stream>>>(p);
-  } else if (D == 64) {
-    if (p.n_units > 0) paged_partial<64><<<(int)p.n_units, kPagedWarps * 32, 0, stream>>>(p);
-    if (merge_blocks > 0) paged_merge<64><<<(int)merge_blocks, 128, 0, stream>>>(p);
-  } else {
+int paged_heads_per_unit(int64_t n_heads, int D) {
+  const int lanes = D / kSlice;           // threads per head
+  const int cap = 256 / lanes;            // heads in a 256-thread CTA
+  const int per_warp = 32 / lanes;        // heads per warp
+  const int64_t h = n_heads < cap ? n_heads : cap;
+  return (int)((h + per_warp - 1) / per_warp * per_warp);  // whole warps
+}
+
+int paged_slots(int D, int max_rows, int heads_per_unit, int num_sms) {
+  const int threads = heads_per_unit * (D / kSlice);
+  int per_sm = 0;
+  cudaError_t e = cudaErrorInvalidValue;
+  if (D == 128)
+    e = max_rows <= 1 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                            &per_sm, paged_partial<128, 1, 4>, threads, 0)
+                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                            &per_sm, paged_partial<128, kPagedRows, 2>, threads, 0);
+  else if (D == 64)
+    e = max_rows <= 1 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                            &per_sm, paged_partial<64, 1, 4>, threads, 0)
+                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                            &per_sm, paged_partial<64, kPagedRows, 2>, threads, 0);
+  if (e != cudaSuccess || per_sm < 1) per_sm = 1;
+  return per_sm * (num_sms > 0 ? num_sms : 1);
+}
+
+cudaError_t launch_paged(int D, int max_rows, const PagedParams& p, cudaStream_t stream) {
+  if (p.n_units > 0x7fffffff || (int64_t)p.n_groups * kPagedRows > 0x7fffffffLL)
     return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
+  if (D == 128) return launch_d<128>(max_rows, p, stream);
+  if (D == 64) return launch_d<64>(max_rows, p, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace fa

@@ -297,50 +297,73 @@ fa_status_t validate_paged(const fa_desc_t* d, const int64_t* prefix, const int6
   return FA_OK;
 }
 
-// Groups in (sequence, head, row block) order, each with the chunks of its
-// visible key range [lo(first row), hi(last row)] (the row intervals are
-// monotone). The chunk length makes about target_units units in all,
-// between 256 and 16384 keys, a multiple of 64.
-void build_paged(const fa_desc_t* d, const std::vector<SeqRec>& recs, int64_t target_units,
-                 std::vector<PagedGroup>* groups, std::vector<PagedUnit>* units) {
+// Groups in (sequence, head, row block) order; the visible key range of a
+// row block is [lo(first row), hi(last row)] (the row intervals are
+// monotone). Units are listed in (sequence, row block, chunk, head run)
+// order; a group's chunks are therefore `runs` units apart. The chunk
+// length is chosen so that all units fit in one wave of `slots` resident
+// CTAs (each span adds at most one short chunk per run), which keeps every
+// SM busy to the end; when there are too many spans for that, chunks of
+// total / (4 slots) keys spread the work over several waves.
+void build_paged(const fa_desc_t* d, const std::vector<SeqRec>& recs, int64_t slots,
+                 int32_t heads_per_unit, std::vector<PagedGroup>* groups,
+                 std::vector<PagedUnit>* units) {
   groups->clear();
   units->clear();
+  const int64_t N = d->N;
+  const int64_t runs = (N + heads_per_unit - 1) / heads_per_unit;
   struct Span { int64_t lo, hi; };
   std::vector<Span> spans;
-  int64_t total = 0;
+  int64_t total = 0;  // keys over all row blocks, times head runs (per run: one unit each)
   for (const SeqRec& s : recs) {
     for (int64_t r0 = 0; r0 < s.sq; r0 += kPagedRows) {
       const int64_t r1 = imin64(r0 + kPagedRows, s.sq) - 1;
       const int64_t lo = imax64(0, row_lo(s, r0));
       const int64_t hi = imin64(int64_t(s.skv) - 1, row_hi(s, r1));
       spans.push_back(Span{lo, hi});
-      if (hi >= lo) total += (hi - lo + 1) * d->N;
+      if (hi >= lo) total += (hi - lo + 1) * runs;
     }
   }
-  int64_t chunk = target_units > 0 ? (total + target_units - 1) / target_units : 256;
-  chunk = imin64(imax64(chunk, 256), 16384);
-  chunk = (chunk + 63) / 64 * 64;
+  int64_t tails = 0;  // spans with keys, times runs: the most short chunks
+  for (const Span& sp : spans)
+    if (sp.hi >= sp.lo) tails += runs;
+  slots = imax64(slots, 1);
+  int64_t chunk = slots > tails ? (total + (slots - tails) - 1) / (slots - tails)
+                                : (total + 4 * slots - 1) / (4 * slots);
+  chunk = imax64(chunk, 64);
   size_t si = 0;
   for (size_t b = 0; b < recs.size(); ++b) {
     const SeqRec& s = recs[b];
-    const size_t first = si;
-    for (int64_t h = 0; h < d->N; ++h) {
-      si = first;
-      for (int64_t r0 = 0; r0 < s.sq; r0 += kPagedRows, ++si) {
-        const Span sp = spans[si];
+    const int64_t nrb = (s.sq + kPagedRows - 1) / kPagedRows;
+    const size_t gbase = groups->size();  // group (b, h, rb) at gbase + h * nrb + rb
+    for (int64_t h = 0; h < N; ++h) {
+      for (int64_t rb = 0; rb < nrb; ++rb) {
         PagedGroup g;
         g.b = (int32_t)b;
         g.h = (int32_t)h;
-        g.row0 = (int32_t)r0;
-        g.nrows = (int32_t)(imin64(r0 + kPagedRows, s.sq) - r0);
-        g.unit0 = (int32_t)units->size();
+        g.row0 = (int32_t)(rb * kPagedRows);
+        g.nrows = (int32_t)(imin64((rb + 1) * kPagedRows, s.sq) - rb * kPagedRows);
+        g.unit0 = 0;
         g.nunits = 0;
-        for (int64_t k0 = sp.lo; k0 <= sp.hi; k0 += chunk) {
-          units->push_back(PagedUnit{(int32_t)groups->size(), (int32_t)k0,
-                                     (int32_t)imin64(k0 + chunk, sp.hi + 1)});
-          ++g.nunits;
-        }
+        g.ustride = (int32_t)runs;
+        g.hslot = (int32_t)(h % heads_per_unit);
         groups->push_back(g);
+      }
+    }
+    for (int64_t rb = 0; rb < nrb; ++rb, ++si) {
+      const Span sp = spans[si];
+      const int32_t first = (int32_t)units->size();
+      const int32_t row0 = (int32_t)(rb * kPagedRows);
+      const int32_t nrows = (int32_t)(imin64((rb + 1) * kPagedRows, s.sq) - rb * kPagedRows);
+      int32_t nchunks = 0;
+      for (int64_t k0 = sp.lo; k0 <= sp.hi; k0 += chunk, ++nchunks)
+        for (int64_t run = 0; run < runs; ++run)
+          units->push_back(PagedUnit{(int32_t)b, row0, nrows, (int32_t)(run * heads_per_unit),
+                                     (int32_t)k0, (int32_t)imin64(k0 + chunk, sp.hi + 1)});
+      for (int64_t h = 0; h < N; ++h) {
+        PagedGroup& g = (*groups)[gbase + h * nrb + rb];
+        g.unit0 = first + (int32_t)(h / heads_per_unit);
+        g.nunits = nchunks;
       }
     }
   }

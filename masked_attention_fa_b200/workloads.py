@@ -7,7 +7,9 @@ can take their inputs from it without sharing any of the method.
 Input recipe (every workload): a CPU ``torch.Generator`` seeded with the
 workload's seed draws, in this order, the varlen lengths (TND workloads
 only), then q, k and v as float32 N(0, 1) which are rounded to bfloat16.
-The scale is 1/sqrt(D).
+The scale is 1/sqrt(D). Paged workloads draw the lengths and the block
+order on the CPU generator and q and the caches on the device the inputs
+are made for (see ``paged_inputs``).
 
 The named workloads follow the shapes of the Ascend "sparseMode参数说明"
 page's scenarios (band, leftUpCausal, right-down band, varlen
@@ -43,6 +45,7 @@ class Workload:
     actual_seq_qlen: Optional[list] = None   # TND cumulative ends (no leading 0)
     actual_seq_kvlen: Optional[list] = None
     scale: Optional[float] = None
+    block_size: Optional[int] = None     # paged K/V caches of this block size (TND queries)
 
     def __post_init__(self):
         if self.scale is None:
@@ -149,10 +152,50 @@ def block_mask(shape, seed: int, block: int = 128, weights=None) -> torch.Tensor
     return out[:, :Sq, :Skv].reshape(*lead, Sq, Skv).contiguous()
 
 
+def decode_lengths(gen: torch.Generator, nseq: int, kv_lo: int, kv_hi: int):
+    """One query token per sequence and Skv_b uniform in [kv_lo, kv_hi]:
+    cumulative end offsets (no leading 0)."""
+    skv = torch.randint(kv_lo, kv_hi + 1, (nseq,), generator=gen)
+    return list(range(1, nseq + 1)), torch.cumsum(skv, 0).tolist()
+
+
+def paged_inputs(w: "Workload", gen: torch.Generator, device="cpu"):
+    """q [T_q, N, D] and paged caches [num_blocks, block_size, N, D] for a
+    TND workload: each sequence's keys fill ceil(Skv_b / block_size) blocks
+    taken in a random order (randperm of the CPU generator `gen`), the rest
+    of a last block is zero; block_table [B, max_blocks] int32 (-1 past a
+    sequence's blocks). q and the cache values (N(0, 1), bf16) are drawn on
+    `device` by a generator of that device seeded with the workload's seed,
+    so a GPU run does not wait for the host to draw gigabytes."""
+    bs = w.block_size
+    lens = w.seq_lens()
+    nblk = [-(-skv // bs) for _, skv in lens]
+    total = sum(nblk)
+    order = torch.randperm(total, generator=gen).to(torch.int32)
+    table = torch.full((len(lens), max(max(nblk), 1)), -1, dtype=torch.int32)
+    nxt = 0
+    for b in range(len(lens)):
+        table[b, :nblk[b]] = order[nxt:nxt + nblk[b]]
+        nxt += nblk[b]
+    dg = torch.Generator(device=device).manual_seed(w.seed)
+    q = torch.randn(w.q_shape(), generator=dg, device=device, dtype=torch.float32).to(torch.bfloat16)
+    k_cache = torch.randn((total, bs, w.N, w.D), generator=dg, device=device, dtype=torch.bfloat16)
+    v_cache = torch.randn((total, bs, w.N, w.D), generator=dg, device=device, dtype=torch.bfloat16)
+    for b, (_, skv) in enumerate(lens):
+        tail = skv - (nblk[b] - 1) * bs
+        if nblk[b] and tail < bs:  # slots past the sequence's last key
+            last = int(table[b, nblk[b] - 1])
+            k_cache[last, tail:] = 0
+            v_cache[last, tail:] = 0
+    return q, k_cache, v_cache, table.to(device)
+
+
 def named_workloads() -> dict:
     """The long-context scenarios, by name."""
     g4 = torch.Generator("cpu").manual_seed(4)
     cu_q, cu_kv = varlen_lengths(g4, 16, 512, 4096, 1024)
+    g6 = torch.Generator("cpu").manual_seed(6)
+    dq, dkv = decode_lengths(g6, 16, 4096, 16384)
     return {
         # band from the top-left via preTokens/nextTokens, with the
         # lower-triangular attenMask the page asks for (causal via band)
@@ -171,6 +214,11 @@ def named_workloads() -> dict:
         # given as an explicit lower-triangular allMask (sparseMode 1)
         "allmask_causal_4k": Workload("allmask_causal_4k", "BNSD", 2, 16, 4096, 4096, 128, 1,
                                       seed=2, mask_kind="SS"),
+        # decode: one query token per sequence against a long context held
+        # in paged caches (blocks of 128 tokens in random order), mode 3
+        "paged_decode_16k": Workload("paged_decode_16k", "TND", 16, 32, dq[-1], dkv[-1], 128, 3,
+                                     seed=6, actual_seq_qlen=dq, actual_seq_kvlen=dkv,
+                                     block_size=128),
     }
 
 
@@ -184,6 +232,11 @@ def make_inputs(w: Workload, device="cpu"):
     if w.layout == "TND" and w.name == "varlen_rightdown_16seq":
         # the lengths were drawn first from the same seed; redraw to advance
         varlen_lengths(g, 16, 512, 4096, 1024)
+    if w.block_size is not None:
+        decode_lengths(g, w.B, 4096, 16384)  # drawn first from the same seed
+        q, k_cache, v_cache, table = paged_inputs(w, g, device)
+        return {"q": q, "k_cache": k_cache, "v_cache": v_cache, "block_table": table,
+                "mask": None}
     q = torch.randn(w.q_shape(), generator=g, dtype=torch.float32).to(torch.bfloat16)
     k = torch.randn(w.kv_shape(), generator=g, dtype=torch.float32).to(torch.bfloat16)
     v = torch.randn(w.kv_shape(), generator=g, dtype=torch.float32).to(torch.bfloat16)
