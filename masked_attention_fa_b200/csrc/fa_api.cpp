@@ -521,6 +521,10 @@ fa_status_t fa_fwd_paged(fa_handle_t h, const void* q, const void* k_cache, cons
   pp.max_blocks = max_blocks;
   pp.n_groups = h->n_groups;
   pp.heads_per_unit = hpu;
+  pp.bs_shift = -1;
+  if ((block_size & (block_size - 1)) == 0)
+    for (int sh = 0; sh < 31; ++sh)
+      if ((1 << sh) == block_size) pp.bs_shift = sh;
   pp.scale_log2 = (float)(d->scale * 1.4426950408889634073599);
   cudaError_t e = launch_paged((int)D, h->paged_rows, pp, stream);
   if (e != cudaSuccess) return cuda_fail(e, "paged kernel launch");

@@ -111,7 +111,8 @@ struct PagedParams {
   int64_t t_q;
   int64_t n_units;
   int32_t n_heads, block_size, max_blocks, n_groups;
-  int32_t heads_per_unit;      // heads one unit (CTA) covers; part is [unit][head][row][D + 2]
+  int32_t heads_per_unit;      // heads one unit (CTA) covers; part is [unit][head][row][D + 4]
+  int32_t bs_shift;            // log2(block_size) when it is a power of two, else -1
   float scale_log2;
 };
 

@@ -106,10 +106,19 @@ __global__ void __launch_bounds__(256) paged_partial(const PagedParams p) {
   const __nv_bfloat16* kc = reinterpret_cast<const __nv_bfloat16*>(p.k_cache);
   const __nv_bfloat16* vc = reinterpret_cast<const __nv_bfloat16*>(p.v_cache);
   const int32_t* table = p.block_table + (int64_t)u.b * p.max_blocks;
+  // Block and offset of key j: a shift and a mask for power-of-two block sizes.
+  const int bs_shift = p.bs_shift;
+  auto block_of = [&](int j) { return bs_shift >= 0 ? j >> bs_shift : j / p.block_size; };
+  auto offset_of = [&](int j) {
+    return bs_shift >= 0 ? j & (p.block_size - 1) : j % p.block_size;
+  };
+  // This thread's elements inside a token row (all heads of a token are adjacent).
+  const int64_t row_elems = (int64_t)p.n_heads * D;
+  const int64_t my_off = (int64_t)h * D + sl * kSlice;
   // The unit's block ids, read once into shared memory (units hold keys, so
   // key1 > key0 and the blocks are table entries [blk0, blk0 + nblk)).
-  const int blk0 = u.key0 / p.block_size;
-  const int nblk = (u.key1 - 1) / p.block_size - blk0 + 1;
+  const int blk0 = block_of(u.key0);
+  const int nblk = block_of(u.key1 - 1) - blk0 + 1;
   const bool staged = nblk <= kTableStage;
   if (staged)
     for (int t = threadIdx.x; t < nblk; t += blockDim.x) sm_blk[t] = __ldg(table + blk0 + t);
@@ -123,13 +132,13 @@ __global__ void __launch_bounds__(256) paged_partial(const PagedParams p) {
       const int j = j0 + e;
       ok[e] = false;
       if (j < u.key1) {
-        const int32_t blk =
-            staged ? sm_blk[j / p.block_size - blk0] : __ldg(table + j / p.block_size);
+        const int bi = block_of(j);
+        const int32_t blk = staged ? sm_blk[bi - blk0] : __ldg(table + bi);
         if (blk >= 0 && (int64_t)blk < p.num_blocks) {
           ok[e] = true;
           if (live) {
-            const int64_t slot = (int64_t)blk * p.block_size + j % p.block_size;
-            const int64_t off = (slot * p.n_heads + h) * D + sl * kSlice;
+            const int64_t slot = (int64_t)blk * p.block_size + offset_of(j);
+            const int64_t off = slot * row_elems + my_off;
             const uint4* ks = reinterpret_cast<const uint4*>(kc + off);
             const uint4* vs = reinterpret_cast<const uint4*>(vc + off);
             kv[e][0] = __ldg(ks);

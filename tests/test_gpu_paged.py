@@ -147,3 +147,43 @@ def test_paged_rejects_bad_arguments_before_device_work():
         attn.paged(q.cuda(), kc.cuda(), vc.cuda(), short.cuda(), cu_q, cu_kv)
     assert e.value.name == "FA_ERR_SHAPE"
     attn.close()
+
+
+def test_paged_decode_workload_full_size_sampled():
+    """The bench's decode workload (16 sequences, 32 heads, 4k-16k cached
+    keys in 128-token blocks, caches drawn on the device) through the call
+    the bench times: sampled (sequence, head) rows against the paged oracle,
+    with the keys of that sequence and head gathered to the host; and two
+    runs give the same bits."""
+    from masked_attention_fa_b200.workloads import make_inputs, named_workloads
+    w = named_workloads()["paged_decode_16k"]
+    inp = make_inputs(w, device="cuda")
+    q, kc, vc, table = (inp[x] for x in ("q", "k_cache", "v_cache", "block_table"))
+    attn = fa.MaskedAttention("TND", w.B, w.N, w.Sq, w.Skv, w.D, w.sparse_mode)
+    try:
+        o1, l1 = attn.paged(q, kc, vc, table, w.actual_seq_qlen, w.actual_seq_kvlen)
+        o2, l2 = attn.paged(q, kc, vc, table, w.actual_seq_qlen, w.actual_seq_kvlen)
+        torch.cuda.synchronize()
+        attn.sync_status()
+    finally:
+        attn.close()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    lens = w.seq_lens()
+    rng = np.random.default_rng(9)
+    for b in sorted({0, w.B - 1, int(rng.integers(0, w.B))}):
+        sq, skv = lens[b]
+        nblk = -(-skv // w.block_size)
+        blocks = table[b, :nblk].long()
+        for h in sorted({0, w.N - 1, int(rng.integers(0, w.N))}):
+            kb = kc[blocks][:, :, h:h + 1].cpu()
+            vb = vc[blocks][:, :, h:h + 1].cpu()
+            q0 = w.actual_seq_qlen[b - 1] if b else 0
+            qb = q[q0:q0 + sq, h:h + 1].cpu()
+            pb = Problem("TND", 1, 1, sq, skv, w.D, sparse_mode=w.sparse_mode, scale=w.scale,
+                         actual_seq_qlen=[sq], actual_seq_kvlen=[skv])
+            o_ref, l_ref = oracle.attention_paged(pb, qb, kb, vb,
+                                                  np.arange(nblk, dtype=np.int32)[None],
+                                                  w.block_size)
+            got = o1[q0:q0 + sq, h:h + 1].float().cpu().double().numpy()
+            gl = l1[h:h + 1, q0:q0 + sq].cpu().double().numpy()
+            assert_close(got, gl, o_ref, l_ref, what=f"sequence {b} head {h}")

@@ -308,3 +308,33 @@ def test_occupancy_output_shapes():
     assert fa.occupancy_shapes(d) == ((3, 1, 2), (3, 1, 4))
     d = fa.make_desc("BNSD", 3, 5, 1, 1, 64, 1, mask_kind="SS")
     assert fa.occupancy_shapes(d) == ((1, 1, 1), (1, 1, 4))
+
+
+def test_paged_entry_point_validates_before_device_work():
+    """fa_fwd_paged rejects bad handles and arguments on the host (the
+    device pointers below are never touched)."""
+    import ctypes
+    lib = fa.load_library()
+    dev = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    I64 = ctypes.c_int64 * 2
+    cu_q, cu_kv = I64(1, 2), I64(40, 70)
+
+    def call(h, q=dev, table=dev, nblk=10, bs=16, maxb=3, cq=cu_q, ckv=cu_kv):
+        return fa.STATUS[lib.fa_fwd_paged(h, q, dev, dev, table, nblk, bs, maxb, None, cq, ckv,
+                                          dev, dev, None)]
+
+    tnd = fa.fa_create(fa.make_desc("TND", 2, 2, 2, 70, 64, 3))
+    bsnd = fa.fa_create(fa.make_desc("BSND", 2, 2, 1, 40, 64, 3))
+    try:
+        assert call(None) == "FA_ERR_NULLPTR"
+        assert call(tnd, table=None) == "FA_ERR_NULLPTR"
+        assert call(bsnd) == "FA_ERR_UNSUPPORTED"
+        assert call(tnd, maxb=2) == "FA_ERR_SHAPE"          # 40 keys need 3 blocks of 16
+        assert call(tnd, bs=0) == "FA_ERR_PARAM_INVALID"
+        assert call(tnd, nblk=0) == "FA_ERR_PARAM_INVALID"
+        assert call(tnd, q=odd) == "FA_ERR_PARAM_INVALID"   # 16-byte alignment
+        assert call(tnd, cq=I64(1, 3)) == "FA_ERR_SHAPE"     # last qlen must equal T_q
+    finally:
+        fa.fa_destroy(tnd)
+        fa.fa_destroy(bsnd)
