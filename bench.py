@@ -62,21 +62,27 @@ def load_peaks():
 
 
 def load_traffic(workload):
-    """Per-launch DRAM bytes (read + write) of the main kernel from the committed
-    ncu summary; None when the kernel source changed since that capture."""
+    """Per-launch DRAM bytes (read + write) of the workload's main kernel from
+    the committed ncu summary; None when that kernel's source changed since
+    the capture (the attention kernel's source unless the record names
+    another)."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    src = os.path.join(ROOT, "masked_attention_fa_b200", "csrc", "fa_kernel_sm100.cu")
     try:
         with open(path) as f:
             rec = json.load(f)
-        with open(src, "rb") as f:
+        entry = rec.get(workload)
+        if entry is None:
+            return None
+        name = entry.get("source", "fa_kernel_sm100.cu")
+        want = entry.get("source_sha256", rec.get("kernel_source_sha256"))
+        with open(os.path.join(ROOT, "masked_attention_fa_b200", "csrc", name), "rb") as f:
             sha = hashlib.sha256(f.read()).hexdigest()
     except (OSError, ValueError):
         return None
-    if rec.get("kernel_source_sha256") != sha or workload not in rec:
+    if sha != want:
         return None
-    return rec[workload].get("dram_bytes_per_launch")
+    return entry.get("dram_bytes_per_launch")
 
 
 class ClockSampler:
