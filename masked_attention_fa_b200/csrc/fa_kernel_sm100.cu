@@ -880,7 +880,9 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
         asm volatile("prefetch.global.L1 [%0];" ::"l"(p.item_tr + 2 * item_index(k + 1)));
     }
     const ItemPlan ip = plan_item<kOcc>(p, idx, it, sr);
-    const TileRange tr = ip.tr[sub];
+    // sub is a run-time value: select, so the plan stays in registers (an
+    // indexed copy would live on the stack, in the SM's small L1).
+    const TileRange tr = sub == 0 ? ip.tr[0] : ip.tr[1];
     const int64_t r0 = (int64_t)it.qblk * kBlockM + sub * kTileM;
     const int i = (int)(r0 + row);  // query row inside the sequence
     const bool row_valid = i < sr.sq;
@@ -1071,7 +1073,7 @@ __device__ void epilogue_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl,
   const int wq = (threadIdx.x >> 5) & 3;
   const int row = wq * 32 + (threadIdx.x & 31);
   const uint32_t lane_bits = (uint32_t)(wq * 32) << 16;
-  uint32_t n_pv[2] = {0u, 0u};  // PVs of each sub-tile so far
+  uint32_t n_pv0 = 0u, n_pv1 = 0u;  // PVs of each sub-tile so far (registers, not an indexed array)
   for (int k = 0;; ++k) {
     const int idx = item_index(k);
     if (idx >= p.n_items) break;
@@ -1089,8 +1091,10 @@ __device__ void epilogue_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl,
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + it.b * p.o_sb +
                             it.h * p.o_sh + ((int64_t)sr.q_off + i) * p.o_st;
       if (tr.hi > tr.lo) {
-        n_pv[sub] += (uint32_t)(tr.hi - tr.lo);
-        if (!wait_warp(&ctl->o_pv[sub], (n_pv[sub] - 1) & 1u, w, kSiteOPv)) return;
+        const uint32_t npv = (sub ? n_pv1 : n_pv0) + (uint32_t)(tr.hi - tr.lo);
+        if (sub) n_pv1 = npv;
+        else n_pv0 = npv;
+        if (!wait_warp(&ctl->o_pv[sub], (npv - 1) & 1u, w, kSiteOPv)) return;
         tc_fence_after();
         const uint32_t tO = tmem + lane_bits + C::col_o(sub);
 #pragma unroll 1
