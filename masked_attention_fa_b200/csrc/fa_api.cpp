@@ -36,7 +36,8 @@ struct fa_handle_s {
   int64_t n_units = 0;
   int32_t paged_rows = 0;  // most query rows in one group
   // device workspace: [error word | pad to 256 B][SeqRec x B][WorkItem x n]
-  // then, for a dense attenMask, the occupancy pre-pass's ranges and classes
+  // [item_tr: 2 x TileRange per item] then, for a dense attenMask, the
+  // occupancy pre-pass's ranges and classes
   void* d_ws = nullptr;
   size_t ws_bytes = 0;
   // pinned staging of the work list and the event of its last upload
@@ -183,10 +184,17 @@ fa_status_t refresh_plan(fa_handle_t h, const int64_t* prefix, const int64_t* cu
   if (items.size() > (size_t)0x7fffffff) return fail(FA_ERR_UNSUPPORTED, "too many work items");
   const size_t seq_bytes = recs.size() * sizeof(SeqRec);
   const size_t item_bytes = items.size() * sizeof(WorkItem);
-  const size_t payload = align_up(seq_bytes, 256) + item_bytes;
   const int64_t planes = mask_planes(&h->desc, has_mask);
+  // Each item's two sub-tile ranges follow the list (item_tr): computed
+  // here from the closed form and uploaded with it, or for a dense mask
+  // written on the device by the rebuild kernel, followed by the pre-pass's
+  // scratch. The kernel then reads a range with one load that does not wait
+  // for the item record (computing it took ~1-2k cycles at each boundary).
+  const size_t tr_off = item_tr_offset((int32_t)recs.size(), (int32_t)items.size());
+  const size_t tr_bytes = items.size() * 2 * sizeof(TileRange);
+  const size_t payload = planes ? align_up(seq_bytes, 256) + item_bytes
+                                : tr_off - kHeaderBytes + tr_bytes;
   const size_t occ = planes ? occupancy_bytes(planes, h->desc.Sq, h->desc.Skv) : 0;
-  // Dense masks: item_tr and the pre-pass's scratch follow the list.
   fa_status_t st = ensure_workspace(
       h, planes ? occupancy_offset((int32_t)recs.size(), (int32_t)items.size()) + occ
                 : kHeaderBytes + payload);
@@ -202,6 +210,16 @@ fa_status_t refresh_plan(fa_handle_t h, const int64_t* prefix, const int64_t* cu
   uint8_t* hs = static_cast<uint8_t*>(h->h_stage);
   std::memcpy(hs, recs.data(), seq_bytes);
   if (item_bytes) std::memcpy(hs + align_up(seq_bytes, 256), items.data(), item_bytes);
+  if (!planes) {  // each item's two sub-tile ranges, from the closed form
+    TileRange* tr = reinterpret_cast<TileRange*>(hs + (tr_off - kHeaderBytes));
+    for (size_t n = 0; n < items.size(); ++n) {
+      const SeqRec& sr = recs[(size_t)items[n].b];
+      for (int st = 0; st < kSubTiles; ++st) {
+        const int64_t r0 = (int64_t)items[n].qblk * kBlockM + st * kTileM;
+        tr[2 * n + st] = r0 < sr.sq ? tile_range(sr, r0) : TileRange{0, 0, 0, 0};
+      }
+    }
+  }
   e = cudaMemcpyAsync(static_cast<uint8_t*>(h->d_ws) + kHeaderBytes, hs, payload,
                       cudaMemcpyHostToDevice, stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(work list)");
@@ -378,6 +396,8 @@ fa_status_t forward(fa_handle_t h, const void* q, const void* k, const void* v,
     if (e != cudaSuccess) return cuda_fail(e, "work list schedule launch");
     p.item_tr = sp.item_tr;
   }
+  if (!has_mask)
+    p.item_tr = reinterpret_cast<const TileRange*>(ws + item_tr_offset(h->n_seqs, h->n_items));
   p.n_items = h->n_items;
   p.tnd = d->layout == FA_TND ? 1 : 0;
   p.scale_log2 = (float)(d->scale * 1.4426950408889634073599);

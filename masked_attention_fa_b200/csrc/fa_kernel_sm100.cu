@@ -415,12 +415,12 @@ struct ItemPlan {
   int nsub;        // sub-tiles with at least one stored row
 };
 
-// Key-tile range of query sub-tile st of item it: the closed-form geometry,
-// or, for a dense attenMask, the range the occupancy pre-pass reduced the
-// mask to. Every role derives its tile sequence from this one function.
-// The kernel is compiled twice: kOcc (dense-mask calls whose pre-pass ran,
-// p.item_tr set) reads the ranges stored beside work item idx, the other
-// computes the closed form, so neither carries the other's code.
+// Key-tile range of query sub-tile st of item it. With kOcc (p.item_tr set:
+// the host's closed-form ranges, or for a dense attenMask the ranges the
+// occupancy pre-pass reduced the mask to) it is read from beside work item
+// idx, one load that does not wait for the item record; without, it is
+// computed from the sequence record (the allocation-free fallback). Every
+// role derives its tile sequence from this one function.
 template <bool kOcc>
 __device__ __forceinline__ TileRange sub_range(const FwdParams& p, int idx, const WorkItem& it,
                                                const SeqRec& s, int st) {
@@ -846,7 +846,9 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // warpgroup that does not visit the tile passes its turn on. At the end of
 // an item it writes the row's log-sum-exp and hands 1/l to the epilogue
 // warpgroup.
-template <int D, bool kOcc>
+// kDense: the dense-mask extras (the next mask line prefetched a tile ahead,
+// 16-byte mask gathers), compiled only into the dense-mask instance.
+template <int D, bool kOcc, bool kDense>
 __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, float* inv_l_sm,
                              uint32_t tmem, uint8_t* sP, int sub, const WaitCtx& w) {
   using C = Cfg<D>;
@@ -862,7 +864,7 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
   // Dense-mask rows start on 16-byte boundaries (base and row stride); the
   // 16-byte gather below is compiled into the dense-mask variant only.
   const bool mask_vec =
-      kOcc && ((reinterpret_cast<uintptr_t>(p.mask) | (uintptr_t)p.m_si) & 15u) == 0;
+      kDense && ((reinterpret_cast<uintptr_t>(p.mask) | (uintptr_t)p.m_si) & 15u) == 0;
   uint32_t s_count = 0;   // S tiles consumed
   uint32_t pv_count = 0;  // P tiles produced = PV MMAs of this sub-tile
   uint32_t turn = 0;      // exponential-unit turns taken
@@ -900,7 +902,7 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
     // Dense-mask variant: the mask line of the next tile that needs it is
     // pulled into L1 a tile ahead, so the gather after S arrives hits L1.
     auto prefetch_mask = [&](int tn) {
-      if constexpr (kOcc) {
+      if constexpr (kDense) {
         if (mrow != nullptr && tn >= tr.lo && tn < tr.hi && !(tn >= tr.full_lo && tn < tr.full_hi))
           asm volatile("prefetch.global.L1 [%0];" ::"l"(mrow + (int64_t)tn * kTileN));
       }
@@ -937,7 +939,7 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
       if (partial && mrow != nullptr) {
         const uint8_t* mt = mrow + (int64_t)t * kTileN;
         bool vec = false;
-        if constexpr (kOcc) vec = mask_vec && (t + 1) * kTileN <= sr.skv;
+        if constexpr (kDense) vec = mask_vec && (t + 1) * kTileN <= sr.skv;
         if (vec) {
           // The whole 128-byte tile row lies inside the mask row and is
           // 16-byte aligned: eight 16-byte loads in flight at once, one bit
@@ -1124,7 +1126,7 @@ __device__ void epilogue_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl,
   }
 }
 
-template <int D, bool kOcc>
+template <int D, bool kOcc, bool kDense>
 __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100(const __grid_constant__ FwdParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -1179,7 +1181,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100(const __grid_constan
 
   if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-    softmax_role<D, kOcc>(p, ctl, inv_l_sm, tmem, sP, warp >> 2, w);
+    softmax_role<D, kOcc, kDense>(p, ctl, inv_l_sm, tmem, sP, warp >> 2, w);
   } else if (warp < 12) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
     epilogue_role<D, kOcc>(p, ctl, inv_l_sm, tmem, w);
@@ -1237,10 +1239,10 @@ bool encode_operand_map(CUtensorMap* tm, const void* base, int64_t D, int64_t S,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool kOcc>
+template <int D, bool kOcc, bool kDense>
 static cudaError_t launch_d(const FwdParams& p, int grid, cudaStream_t stream, const char** why) {
   using C = dev::Cfg<D>;
-  auto kern = dev::fa_fwd_sm100<D, kOcc>;
+  auto kern = dev::fa_fwd_sm100<D, kOcc, kDense>;
   static bool configured = false;
   static bool regs_ok = false;
   if (!configured) {
@@ -1265,11 +1267,18 @@ static cudaError_t launch_d(const FwdParams& p, int grid, cudaStream_t stream, c
 
 cudaError_t launch_fwd(int D, const FwdParams& p, int grid, cudaStream_t stream,
                        const char** why) {
+  // Three instances per head dim: ranges beside the items with and without
+  // the dense-mask extras, and ranges from the closed form (no item_tr).
   const bool occ = p.item_tr != nullptr;
-  if (D == 128) return occ ? launch_d<128, true>(p, grid, stream, why)
-                           : launch_d<128, false>(p, grid, stream, why);
-  if (D == 64) return occ ? launch_d<64, true>(p, grid, stream, why)
-                          : launch_d<64, false>(p, grid, stream, why);
+  const bool dense = occ && p.mask != nullptr && p.m_si > 0;
+  if (D == 128)
+    return dense ? launch_d<128, true, true>(p, grid, stream, why)
+                 : occ ? launch_d<128, true, false>(p, grid, stream, why)
+                       : launch_d<128, false, false>(p, grid, stream, why);
+  if (D == 64)
+    return dense ? launch_d<64, true, true>(p, grid, stream, why)
+                 : occ ? launch_d<64, true, false>(p, grid, stream, why)
+                       : launch_d<64, false, false>(p, grid, stream, why);
   if (why) *why = "unsupported head dim";
   return cudaErrorInvalidValue;
 }

@@ -268,6 +268,25 @@ extern "C" fa_status_t fa_fwd_noalloc(const fa_desc_t* desc, const void* q, cons
     p.m_sb = (d->mask_kind == FA_MASK_SS) ? 0 : (d->mask_kind == FA_MASK_B1SS ? plane : d->N * plane);
     p.m_sh = (d->mask_kind == FA_MASK_BNSS) ? plane : 0;
   }
+  if (!has_mask && n > 0) {
+    // Each item's two sub-tile ranges beside the list when they fit, as the
+    // handle path keeps them (else the kernel computes them per item).
+    const size_t tr_off = round256(need);
+    if (tr_off + n * 2 * sizeof(TileRange) <= kNoAllocScratchBytes) {
+      TileRange* tr = reinterpret_cast<TileRange*>(g_host_image + tr_off);
+      for (size_t m = 0; m < n; ++m) {
+        const SeqRec& sr = recs[items[m].b];
+        for (int st = 0; st < kSubTiles; ++st) {
+          const int64_t r0 = (int64_t)items[m].qblk * kBlockM + st * kTileM;
+          tr[2 * m + st] = r0 < sr.sq ? tile_range(sr, r0) : TileRange{0, 0, 0, 0};
+        }
+      }
+      e = cudaMemcpyAsync(dscr + tr_off, g_host_image + tr_off, n * 2 * sizeof(TileRange),
+                          cudaMemcpyHostToDevice, stream);
+      if (e != cudaSuccess) return cuda_err(e, "cudaMemcpyAsync(item ranges)");
+      p.item_tr = reinterpret_cast<const TileRange*>(dscr + tr_off);
+    }
+  }
   if (has_mask && n > 0) {
     // The occupancy pre-pass and the device-side list rebuild run when their
     // scratch (each item's ranges, the pre-pass's table and classes) fits
