@@ -515,7 +515,7 @@ def main():
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": traffic,
                     "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
-                    "kernel": f"fa_fwd_sm100<{w.D}, {'true' if dense else 'false'}>",
+                    "kernel": f"fa_fwd_sm100<{w.D}, true, {'true' if dense else 'false'}>",
                     "kernel_ms": kern_ms}
         if paged:
             # A few query rows per sequence: every cached K/V byte is used for a
