@@ -85,3 +85,57 @@ def test_named_workload_sampled_rows(name):
     le = np.concatenate(lerrs)
     assert e.max() <= TOL_MAX_O and e.mean() <= TOL_MEAN_O, (name, e.max(), e.mean())
     assert le.max() <= TOL_LSE, (name, le.max())
+
+
+def test_one_sequence_of_a_million_tokens():
+    """BSND, one sequence of 2^20 query rows and keys, causal (mode 2), D=64:
+    every index that could overflow 32 bits at this length (token offsets
+    times strides, tile and item counts) is exercised. Sampled rows, the
+    last one seeing all 2^20 keys, against the fp64 oracle."""
+    S, D = 1 << 20, 64
+    g = torch.Generator(device="cuda").manual_seed(77)
+    q = torch.randn(1, S, 1, D, generator=g, device="cuda").to(torch.bfloat16)
+    k = torch.randn(1, S, 1, D, generator=g, device="cuda").to(torch.bfloat16)
+    v = torch.randn(1, S, 1, D, generator=g, device="cuda").to(torch.bfloat16)
+    attn = fa.MaskedAttention("BSND", 1, 1, S, S, D, 2)
+    o, lse = attn(q, k, v)
+    torch.cuda.synchronize()
+    attn.sync_status()
+    attn.close()
+    assert torch.isfinite(o.float()).all()
+    rows = [0, 1, 255, 256, 65535, 65536, S // 2 + 3, S - 129, S - 1]
+    pb = Problem("BSND", 1, 1, S, S, D, sparse_mode=2)
+    o_ref, l_ref = oracle.attention_rows(pb, q.cpu(), k.cpu(), v.cpu(), [(0, 0, i) for i in rows])
+    got = o[0, rows, 0].float().cpu().double().numpy()
+    gl = lse[0, 0, rows].cpu().double().numpy()
+    assert np.abs(got - o_ref).max() <= TOL_MAX_O
+    assert np.abs(gl - l_ref).max() <= TOL_LSE
+
+
+def test_thousands_of_tiny_varlen_sequences():
+    """TND with 3000 sequences of 0-9 query rows and 0-12 keys (rightDownCausal:
+    many rows see no key, many sequences have none), compared in full."""
+    rng = np.random.default_rng(78)
+    lq = rng.integers(0, 10, size=3000)
+    lk = rng.integers(0, 13, size=3000)
+    cu_q, cu_k = np.cumsum(lq).tolist(), np.cumsum(lk).tolist()
+    N, D = 2, 128
+    g = torch.Generator().manual_seed(78)
+    q = torch.randn(cu_q[-1], N, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(cu_k[-1], N, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(cu_k[-1], N, D, generator=g).to(torch.bfloat16)
+    attn = fa.MaskedAttention("TND", 3000, N, cu_q[-1], cu_k[-1], D, 3)
+    o, lse = attn(q.cuda(), k.cuda(), v.cuda(), actual_seq_qlen=cu_q, actual_seq_kvlen=cu_k)
+    torch.cuda.synchronize()
+    attn.sync_status()
+    attn.close()
+    pb = Problem("TND", 3000, N, cu_q[-1], cu_k[-1], D, sparse_mode=3, actual_seq_qlen=cu_q,
+                 actual_seq_kvlen=cu_k)
+    o_ref, l_ref = oracle.attention(pb, q, k, v)
+    o = o.float().cpu().double().numpy()
+    lse = lse.cpu().double().numpy()
+    dead = np.isneginf(l_ref)
+    assert np.array_equal(np.isneginf(lse), dead)
+    assert np.abs(o - o_ref).max() <= TOL_MAX_O
+    assert np.abs(o - o_ref).mean() <= TOL_MEAN_O
+    assert np.abs(lse[~dead] - l_ref[~dead]).max() <= TOL_LSE
