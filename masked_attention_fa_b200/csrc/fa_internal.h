@@ -46,7 +46,7 @@ struct WorkItem {
   int32_t b;
   int32_t h;
   int32_t qblk;
-  int32_t cost;  // non-empty KV tiles over both sub-tiles (LPT key)
+  int32_t cost;  // longest-first key: lpt_key on the host, the tile sum in the device rebuild
 };
 static_assert(sizeof(WorkItem) == 16, "WorkItem layout");
 

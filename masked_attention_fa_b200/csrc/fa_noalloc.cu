@@ -214,11 +214,8 @@ extern "C" fa_status_t fa_fwd_noalloc(const fa_desc_t* desc, const void* q, cons
     if (s.sq <= 0) continue;
     const int32_t nblk = (s.sq + kBlockM - 1) / kBlockM;
     for (int32_t qb = 0; qb < nblk; ++qb) {
-      int32_t cost = 0;
-      for (int sub = 0; sub < kSubTiles; ++sub) {
-        const TileRange t = tile_range(s, (int64_t)qb * kBlockM + sub * kTileM);
-        cost += t.hi > t.lo ? t.hi - t.lo : 0;
-      }
+      const int32_t cost = lpt_key(tile_range(s, (int64_t)qb * kBlockM),
+                                   tile_range(s, (int64_t)qb * kBlockM + kTileM));
       for (int64_t h = 0; h < desc->N; ++h) items[n++] = WorkItem{(int32_t)b, (int32_t)h, qb, cost};
     }
   }

@@ -250,10 +250,9 @@ std::vector<SeqRec> decode_geometry(const fa_desc_t* d, const int64_t* prefix,
   return recs;
 }
 
-static int32_t tiles_of(const TileRange& t) { return t.hi > t.lo ? t.hi - t.lo : 0; }
 
 // One item per (sequence, head, 256-row block). Items are sorted by
-// descending cost (longest-processing-time first), ties in index order.
+// descending lpt_key (longest-processing-time first), ties in index order.
 std::vector<WorkItem> build_items(const fa_desc_t* d, const std::vector<SeqRec>& recs) {
   std::vector<WorkItem> items;
   for (int64_t b = 0; b < d->B; ++b) {
@@ -261,9 +260,8 @@ std::vector<WorkItem> build_items(const fa_desc_t* d, const std::vector<SeqRec>&
     if (s.sq <= 0) continue;
     const int32_t nblk = (s.sq + kBlockM - 1) / kBlockM;
     for (int32_t qb = 0; qb < nblk; ++qb) {
-      int32_t cost = 0;
-      for (int st = 0; st < kSubTiles; ++st)
-        cost += tiles_of(tile_range(s, (int64_t)qb * kBlockM + st * kTileM));
+      const int32_t cost = lpt_key(tile_range(s, (int64_t)qb * kBlockM),
+                                   tile_range(s, (int64_t)qb * kBlockM + kTileM));
       for (int64_t h = 0; h < d->N; ++h)
         items.push_back(WorkItem{(int32_t)b, (int32_t)h, qb, cost});
     }
