@@ -154,6 +154,20 @@ def workload_args(w):
     return arrays
 
 
+def kernel_label(w, dense, dev):
+    """The attention kernel instance a call of the workload runs: dense-mask
+    extras, and claimed work for closed-form lists of at least
+    fa.CLAIM_MIN_ITEMS_PER_CTA items per SM."""
+    import torch
+    import masked_attention_fa_b200 as fa
+    d = fa.make_desc(w.layout, w.B, w.N, w.Sq, w.Skv, w.D, w.sparse_mode, w.pre_tokens,
+                     w.next_tokens, w.scale, w.mask_kind)
+    items = fa.fa_plan_stats(d, has_mask=dense, **workload_args(w))[0]
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    claim = (not dense) and items >= fa.CLAIM_MIN_ITEMS_PER_CTA * sms
+    return f"fa_fwd_sm100<{w.D}, true, {'true' if dense else 'false'}, {'true' if claim else 'false'}>"
+
+
 def visible_pairs(w, has_mask, mask_host=None):
     """Visible pairs of the workload from the library's geometry (closed-form
     row intervals); dense-mask workloads count the mask on the host."""
@@ -515,7 +529,7 @@ def main():
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": traffic,
                     "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
-                    "kernel": f"fa_fwd_sm100<{w.D}, true, {'true' if dense else 'false'}>",
+                    "kernel": kernel_label(w, dense, dev),
                     "kernel_ms": kern_ms}
         if paged:
             # A few query rows per sequence: every cached K/V byte is used for a

@@ -24,7 +24,10 @@
  *  - Results are bitwise deterministic: every output row is produced by one
  *    CTA, visiting its key tiles in a fixed order (no split-K atomics), as
  *    the aclnnScatterPaKvCache page's "确定性计算" note asks of that op.
- *  - A handle is not thread-safe; distinct handles are independent.
+ *  - A handle is not thread-safe; distinct handles are independent. The
+ *    calls of one handle must not overlap on the GPU (enqueue them on one
+ *    stream, or order them with events): they share its device workspace,
+ *    including the counter from which long work lists are claimed.
  */
 #ifndef FA_B200_FA_H
 #define FA_B200_FA_H
@@ -133,6 +136,13 @@ fa_status_t fa_create(const fa_desc_t* desc, fa_handle_t* out);
  * without reading it, then a one-block kernel that rebuilds the work list
  * from the pre-pass's ranges, longest item first by its real number of key
  * tiles; fa_fwd_with_ranges skips the pre-pass but not the rebuild.
+ *
+ * Work distribution: items (sequence, head, 256 query rows) are sorted
+ * longest first. A closed-form call whose list holds at least 8 items per
+ * SM lets each CTA claim its next item from a counter in the workspace
+ * while it loads its current one (the last CTA resets it); otherwise each
+ * CTA takes a fixed share. Every output row is produced by one CTA either
+ * way, so results do not depend on which CTA computed them.
  *
  * Asynchronous: returns once the kernel is enqueued. The host arrays are
  * read during the call only. Device-side problems (a wait that gave up) are

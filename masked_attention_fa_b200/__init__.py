@@ -126,6 +126,12 @@ def _check(status):
         raise FaError(status, msg)
 
 
+# Work-list size per SM from which closed-form calls claim their items at
+# run time (the library's kClaimMinItemsPerCta; used to name the kernel
+# instance a call runs).
+CLAIM_MIN_ITEMS_PER_CTA = 8
+
+
 def make_desc(layout, B, N, Sq, Skv, D, sparse_mode=0, pre_tokens=0, next_tokens=0, scale=None,
               mask_kind=None) -> fa_desc_t:
     lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)

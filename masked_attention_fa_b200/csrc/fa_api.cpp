@@ -35,7 +35,8 @@ struct fa_handle_s {
   int32_t n_groups = 0;
   int64_t n_units = 0;
   int32_t paged_rows = 0;  // most query rows in one group
-  // device workspace: [error word | pad to 256 B][SeqRec x B][WorkItem x n]
+  // device workspace: [error word | claim counter at 128 | claim_done at 192 |
+  // pad to 256 B][SeqRec x B][WorkItem x n]
   // [item_tr: 2 x TileRange per item] then, for a dense attenMask, the
   // occupancy pre-pass's ranges and classes
   void* d_ws = nullptr;
@@ -56,6 +57,7 @@ struct fa_handle_s {
 namespace {
 
 constexpr size_t kHeaderBytes = 256;
+constexpr size_t kClaimOffset = 128;  // two work-claim counters, 64 bytes apart
 
 bool env_flag(const char* name) {
   const char* v = std::getenv(name);
@@ -399,6 +401,13 @@ fa_status_t forward(fa_handle_t h, const void* q, const void* k, const void* v,
   if (!has_mask)
     p.item_tr = reinterpret_cast<const TileRange*>(ws + item_tr_offset(h->n_seqs, h->n_items));
   p.n_items = h->n_items;
+  // Closed-form lists (descending lpt_key: items without a key tile last)
+  // with many items per CTA are claimed at run time.
+  if (!has_mask && (int64_t)h->n_items >= (int64_t)kClaimMinItemsPerCta * h->num_sms &&
+      h->n_items < 0x7fff0000) {
+    p.claim = reinterpret_cast<unsigned int*>(ws + kClaimOffset);
+    p.claim_done = reinterpret_cast<unsigned int*>(ws + kClaimOffset + 64);
+  }
   p.tnd = d->layout == FA_TND ? 1 : 0;
   p.scale_log2 = (float)(d->scale * 1.4426950408889634073599);
   p.debug_flags = h->debug_flags;

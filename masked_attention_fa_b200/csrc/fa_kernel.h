@@ -33,12 +33,29 @@ struct __align__(64) FwdParams {
   // Dense-mask calls (or null): the key-tile ranges of sub-tiles 0 and 1
   // of work item idx are item_tr[2 idx] and item_tr[2 idx + 1].
   const TileRange* item_tr;
+  // Work claiming (or null: each CTA takes the fixed snake of positions
+  // c, 2G-1-c, 2G+c, ... of the list). With a counter, CTA c starts at
+  // position c and every later item is the next unclaimed position G + n,
+  // n from atomicAdd(claim, 1), taken while the CTA still loads its current
+  // item; the last CTA to finish sets claim and claim_done back to 0. Needs
+  // every item without a key tile after every item with one (a list sorted
+  // by descending cost), and calls that do not overlap on the GPU.
+  unsigned int* claim;
+  unsigned int* claim_done;
   int32_t n_items;
   int32_t tnd;             // packed tokens: TMA batch coordinate 0, token = offset + row
   float scale_log2;        // scale * log2(e)
   uint32_t debug_flags;
   uint64_t timeout_ns;     // limit of every device-side wait
 };
+
+// Closed-form calls claim their items at run time (FwdParams::claim, a
+// kernel instance of its own) when the list holds at least this many items
+// per CTA: claims even out the differences in speed between SMs and the
+// error of the cost key, which the fixed snake cannot, at a small cost per
+// item. With fewer, each CTA's share is a few long items that the snake
+// balances as well.
+constexpr int kClaimMinItemsPerCta = 8;
 
 enum DebugFlags : uint32_t {
   // The TMA warp of CTA 0 never loads its first Q tile, so the MMA warp's

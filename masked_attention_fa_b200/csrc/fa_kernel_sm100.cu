@@ -59,8 +59,17 @@ constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 
 enum WaitSite : uint32_t {
   kSiteQEmpty = 1, kSiteKvEmpty = 2, kSiteQFull = 3, kSiteKvFull = 4, kSitePFull = 5,
   kSiteSFull = 6, kSiteOPv = 7, kSiteDrain = 8, kSiteSFree = 9, kSiteOFree = 10,
-  kSiteMufu = 11, kSiteEpi = 12, kSiteStatFree = 13,
+  kSiteMufu = 11, kSiteEpi = 12, kSiteStatFree = 13, kSiteIdxFull = 14, kSiteIdxEmpty = 15,
 };
+
+// Claimed work (the kClaim instance): the TMA thread claims the CTA's items
+// and passes their indices to the other roles through a ring of kIdxSlots
+// shared-memory slots, read by the QK and PV threads, the 8 softmax warps
+// and the 4 epilogue warps. A claim is taken kClaimLead key tiles before
+// the TMA thread's last loads of its current item.
+constexpr int kIdxSlots = 8;
+constexpr int kIdxReaders = 14;
+constexpr int kClaimLead = 2;
 
 template <int D>
 struct Cfg {
@@ -105,6 +114,9 @@ struct Ctl {
   uint64_t drain[2];  // one per MMA-issuing thread
   uint32_t tmem_base;
   volatile int abort_flag;
+  uint64_t idx_full[kIdxSlots];   // slot holds the index of this CTA's next item
+  uint64_t idx_empty[kIdxSlots];  // every reader has taken it
+  int idx_ring[kIdxSlots];
 };
 
 // ----------------------------------------------------------------- basics
@@ -333,6 +345,42 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, ok);
 }
 
+// k-th item index of this CTA into the ring (TMA thread). The arrive
+// releases the store; the readers' wait acquires it.
+template <int NS>
+__device__ __forceinline__ bool idx_publish(Ctl<NS>* ctl, int k, int idx, const WaitCtx& w) {
+  const int slot = k % kIdxSlots;
+  if (k >= kIdxSlots &&
+      !wait_bounded(&ctl->idx_empty[slot], ((k / kIdxSlots) - 1) & 1u, w, kSiteIdxEmpty))
+    return false;
+  ctl->idx_ring[slot] = idx;
+  mbar_arrive(&ctl->idx_full[slot]);
+  return true;
+}
+
+// k-th item index of this CTA (one thread); INT_MAX, which ends every role's
+// list, when the wait gave up.
+template <int NS>
+__device__ __forceinline__ int idx_take(Ctl<NS>* ctl, int k, const WaitCtx& w) {
+  const int slot = k % kIdxSlots;
+  if (!wait_bounded(&ctl->idx_full[slot], (k / kIdxSlots) & 1u, w, kSiteIdxFull))
+    return 0x7fffffff;
+  const int idx = *reinterpret_cast<volatile int*>(&ctl->idx_ring[slot]);
+  mbar_arrive(&ctl->idx_empty[slot]);
+  return idx;
+}
+
+// The same for a whole warp: one release per warp, after every lane read.
+template <int NS>
+__device__ __forceinline__ int idx_take_warp(Ctl<NS>* ctl, int k, const WaitCtx& w) {
+  const int slot = k % kIdxSlots;
+  if (!wait_warp(&ctl->idx_full[slot], (k / kIdxSlots) & 1u, w, kSiteIdxFull)) return 0x7fffffff;
+  const int idx = *reinterpret_cast<volatile int*>(&ctl->idx_ring[slot]);
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&ctl->idx_empty[slot]);
+  return idx;
+}
+
 // ----------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -467,7 +515,10 @@ __device__ __forceinline__ bool active(const TileRange& t, int j) { return j >= 
 // first K (or the end of the work list). A Q tile is loaded once its buffer
 // is released by the last QK of the previous item on that sub-tile; placing
 // Q1 after the first K keeps a late Q1 release from holding back K.
-template <int D, bool kOcc>
+// With kClaim this thread also takes the CTA's items: it publishes the index
+// of each into the ring, the next one once its claim returns, before the
+// loads the other roles need to finish the current item.
+template <int D, bool kOcc, bool kClaim>
 __device__ void load_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint8_t* sQ,
                           uint8_t* sKV, const WaitCtx& w) {
   using C = Cfg<D>;
@@ -506,6 +557,7 @@ __device__ void load_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint8_t
   struct PendingV {
     int row, h, bc;
   } pend{0, -1, 0};
+  if constexpr (!kClaim) {
   for (int k = 0; ok; ++k) {
     const int idx = item_index(k);
     if (idx >= p.n_items) break;
@@ -525,6 +577,53 @@ __device__ void load_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint8_t
       if (ok) ok = load_kv(&p.tm_v, sr.kv_off + t * kTileN, it.h, bc);
     }
     pend = PendingV{sr.kv_off + (ip.hi - 1) * kTileN, it.h, bc};
+  }
+  } else {
+  int idx = item_index(0);
+  ok = idx_publish(ctl, 0, idx, w);
+  for (int k = 0; ok && idx < p.n_items; ++k) {
+    const WorkItem it = p.items[idx];
+    const SeqRec sr = p.seqs[it.b];
+    const ItemPlan ip = plan_item<kOcc>(p, idx, it, sr);
+    // Items without a key tile come last: the first one this CTA claims ends
+    // its loads, so the last V goes now, not after the remaining claims (the
+    // PV thread needs it before the other roles can finish the current item
+    // and free the ring slots those claims need).
+    if (ip.hi <= ip.lo && pend.h >= 0) {
+      ok = load_kv(&p.tm_v, pend.row, pend.h, pend.bc);
+      pend.h = -1;
+    }
+    unsigned int ticket = 0u;
+    bool claimed = false;
+    if (ok && ip.hi > ip.lo) {
+      const int bc = p.tnd ? 0 : it.b;
+      const int claim_at = max(ip.lo, ip.hi - 1 - kClaimLead);
+      if (ip.tr[0].hi > ip.tr[0].lo) ok = load_q(it, sr, 0, bc);
+      if (ok) ok = load_kv(&p.tm_k, sr.kv_off + ip.lo * kTileN, it.h, bc);
+      if (ok && ip.tr[1].hi > ip.tr[1].lo) ok = load_q(it, sr, 1, bc);
+      if (ok && pend.h >= 0) ok = load_kv(&p.tm_v, pend.row, pend.h, pend.bc);
+      for (int t = ip.lo; t + 1 < ip.hi && ok; ++t) {
+        // The claim's result is first used after this loop, so its round
+        // trip overlaps the item's last loads.
+        if (!claimed && t >= claim_at) {
+          ticket = atomicAdd(p.claim, 1u);
+          claimed = true;
+        }
+        ok = load_kv(&p.tm_k, sr.kv_off + (t + 1) * kTileN, it.h, bc);
+        if (ok) ok = load_kv(&p.tm_v, sr.kv_off + t * kTileN, it.h, bc);
+      }
+      pend = PendingV{sr.kv_off + (ip.hi - 1) * kTileN, it.h, bc};
+    }
+    if (!ok) break;
+    if (!claimed) ticket = atomicAdd(p.claim, 1u);
+    const int next = (int)(gridDim.x + ticket);  // at most n_items + gridDim.x - 1
+    if (next < p.n_items) {
+      asm volatile("prefetch.global.L1 [%0];" ::"l"(p.items + next));
+      if constexpr (kOcc) asm volatile("prefetch.global.L1 [%0];" ::"l"(p.item_tr + 2 * next));
+    }
+    ok = idx_publish(ctl, k + 1, next, w);
+    idx = next;
+  }
   }
   if (ok && pend.h >= 0) ok = load_kv(&p.tm_v, pend.row, pend.h, pend.bc);
   if (!ok) {
@@ -590,24 +689,36 @@ struct MmaPlan {
   int pos;
 };
 
-// Next item of this CTA with at least one key tile, from position k on.
+// Key-tile ranges of item idx; false when it has no key tile.
 template <bool kOcc>
-__device__ __forceinline__ bool next_item(const FwdParams& p, int& k, MmaPlan& mp) {
+__device__ __forceinline__ bool mma_plan(const FwdParams& p, int idx, MmaPlan& mp) {
+  const WorkItem it = p.items[idx];
+  const ItemPlan ip = plan_item<kOcc>(p, idx, it, p.seqs[it.b]);
+  if (ip.hi <= ip.lo) return false;
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    mp.lo[s] = ip.tr[s].lo;
+    mp.hi[s] = ip.tr[s].hi;
+  }
+  mp.lo[2] = ip.lo;
+  mp.hi[2] = ip.hi;
+  return true;
+}
+
+// Next item of this CTA with at least one key tile, from position k on:
+// computed from the snake, or (kRing) read from the index ring, every slot
+// up to the one that ends the list.
+template <bool kOcc, bool kRing, int NS>
+__device__ __forceinline__ bool next_item(const FwdParams& p, Ctl<NS>* ctl, const WaitCtx& w,
+                                          int& k, MmaPlan& mp) {
   for (;; ++k) {
-    const int idx = item_index(k);
+    int idx;
+    if constexpr (kRing) idx = idx_take(ctl, k, w);
+    else idx = item_index(k);
     if (idx >= p.n_items) return false;
-    const WorkItem it = p.items[idx];
-    const ItemPlan ip = plan_item<kOcc>(p, idx, it, p.seqs[it.b]);
-    if (ip.hi > ip.lo) {
+    if (mma_plan<kOcc>(p, idx, mp)) {
       mp.pos = k;
       ++k;
-#pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        mp.lo[s] = ip.tr[s].lo;
-        mp.hi[s] = ip.tr[s].hi;
-      }
-      mp.lo[2] = ip.lo;
-      mp.hi[2] = ip.hi;
       return true;
     }
   }
@@ -631,7 +742,7 @@ __device__ __forceinline__ uint32_t ring_v(uint32_t g, bool last) {
 // It runs ahead of the P.V stream (another thread), limited only by the
 // softmax releasing S, so the scores of the next tile, also across item
 // boundaries, are ready when the softmax wants them.
-template <int D, bool kOcc>
+template <int D, bool kOcc, bool kClaim>
 __device__ void qk_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t tmem,
                         const uint8_t* sQ, const uint8_t* sKV, const WaitCtx& w) {
   using C = Cfg<D>;
@@ -642,7 +753,7 @@ __device__ void qk_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
   bool ok = true;
   int k = 0;
   MmaPlan cur;
-  while (ok && next_item<kOcc>(p, k, cur)) {
+  while (ok && next_item<kOcc, kClaim>(p, ctl, w, k, cur)) {
     bool q_ready[2] = {false, false};
     for (int t = cur.lo[2]; t < cur.hi[2] && ok; ++t, ++g) {
       const uint32_t r = ring_k(g);
@@ -686,7 +797,7 @@ __device__ void qk_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
 // the commit after it tells the softmax that O_s is updated and that the P
 // buffer may be rewritten. The first PV of an item overwrites O_s, so it
 // waits until the epilogue has read O_s of the previous item that had one.
-template <int D, bool kOcc>
+template <int D, bool kOcc, bool kClaim>
 __device__ void pv_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t tmem,
                         const uint8_t* sP, const uint8_t* sKV, const WaitCtx& w) {
   using C = Cfg<D>;
@@ -697,13 +808,29 @@ __device__ void pv_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
   bool ok = true;
   int k = 0;
   MmaPlan cur;
-  bool have = next_item<kOcc>(p, k, cur);
+  bool have = next_item<kOcc, kClaim>(p, ctl, w, k, cur);
+  bool at_end = !have;  // kClaim: the slot that ends the list has been read
   while (ok && have) {
     MmaPlan nxt;
-    const bool have_next = next_item<kOcc>(p, k, nxt);
+    bool have_next = false;
+    if constexpr (!kClaim) have_next = next_item<kOcc, false>(p, ctl, w, k, nxt);
     bool first[2] = {true, true};
     for (int t = cur.lo[2]; t < cur.hi[2] && ok; ++t, ++g) {
-      const uint32_t r = ring_v(g, !have_next && t + 1 == cur.hi[2]);
+      const bool last_t = t + 1 == cur.hi[2];
+      if constexpr (kClaim) {
+        // A claimed next item is known once the TMA thread's claim returns,
+        // published before it loads this item's last V: look at one slot at
+        // the last key tile. Items without a key tile come last, so one of
+        // them (or the end of the list) ends this thread's MMAs; the slots
+        // after it are read once those are issued.
+        if (last_t) {
+          const int nidx = idx_take(ctl, k, w);
+          ++k;
+          if (nidx >= p.n_items) at_end = true;
+          else have_next = mma_plan<kOcc>(p, nidx, nxt);
+        }
+      }
+      const uint32_t r = ring_v(g, !have_next && last_t);
       if (!wait_bounded(&ctl->kv_full[r % NS], (r / NS) & 1u, w, kSiteKvFull)) {
         ok = false;
         break;
@@ -735,6 +862,11 @@ __device__ void pv_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
     }
     cur = nxt;
     have = have_next;
+  }
+  if constexpr (kClaim) {
+    if (ok && !at_end)
+      while (idx_take(ctl, k++, w) < p.n_items) {
+      }
   }
   mma_commit(&ctl->drain[1]);
   wait_bounded(&ctl->drain[1], 0u, w, kSiteDrain, false);
@@ -848,7 +980,7 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // warpgroup.
 // kDense: the dense-mask extras (the next mask line prefetched a tile ahead,
 // 16-byte mask gathers), compiled only into the dense-mask instance.
-template <int D, bool kOcc, bool kDense>
+template <int D, bool kOcc, bool kDense, bool kClaim>
 __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, float* inv_l_sm,
                              uint32_t tmem, uint8_t* sP, int sub, const WaitCtx& w) {
   using C = Cfg<D>;
@@ -870,13 +1002,16 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
   uint32_t turn = 0;      // exponential-unit turns taken
   bool ok = true;
   for (int k = 0; ok; ++k) {
-    const int idx = item_index(k);
+    int idx;
+    if constexpr (kClaim) idx = idx_take_warp(ctl, k, w);
+    else idx = item_index(k);
     if (idx >= p.n_items) break;
     const WorkItem it = p.items[idx];
     const SeqRec sr = p.seqs[it.b];
     // The next item's record is read at the item boundary, on the critical
-    // path of the exponential-unit turns: pull it into L1 now.
-    if (lane == 0 && item_index(k + 1) < p.n_items) {
+    // path of the exponential-unit turns: pull it into L1 now (a claimed
+    // item is prefetched by the TMA thread once its claim returns).
+    if (!kClaim && lane == 0 && item_index(k + 1) < p.n_items) {
       asm volatile("prefetch.global.L1 [%0];" ::"l"(p.items + item_index(k + 1)));
       if constexpr (kOcc)
         asm volatile("prefetch.global.L1 [%0];" ::"l"(p.item_tr + 2 * item_index(k + 1)));
@@ -1068,7 +1203,7 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
 // item and sub-tile, once the softmax has handed over 1/l and the item's last
 // PV is done, O_s / l -> bf16 rows in global memory (zeros for rows that see
 // no key); 1/l is released as soon as it is read, O_s once it is read.
-template <int D, bool kOcc>
+template <int D, bool kOcc, bool kClaim>
 __device__ void epilogue_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl,
                               const float* inv_l_sm, uint32_t tmem, const WaitCtx& w) {
   using C = Cfg<D>;
@@ -1077,7 +1212,9 @@ __device__ void epilogue_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl,
   const uint32_t lane_bits = (uint32_t)(wq * 32) << 16;
   uint32_t n_pv0 = 0u, n_pv1 = 0u;  // PVs of each sub-tile so far (registers, not an indexed array)
   for (int k = 0;; ++k) {
-    const int idx = item_index(k);
+    int idx;
+    if constexpr (kClaim) idx = idx_take_warp(ctl, k, w);
+    else idx = item_index(k);
     if (idx >= p.n_items) break;
     const WorkItem it = p.items[idx];
     const SeqRec sr = p.seqs[it.b];
@@ -1126,7 +1263,7 @@ __device__ void epilogue_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl,
   }
 }
 
-template <int D, bool kOcc, bool kDense>
+template <int D, bool kOcc, bool kDense, bool kClaim>
 __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100(const __grid_constant__ FwdParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -1162,6 +1299,12 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100(const __grid_constan
     }
     mbar_init(&ctl->drain[0], 1);
     mbar_init(&ctl->drain[1], 1);
+    if constexpr (kClaim) {
+      for (int r = 0; r < kIdxSlots; ++r) {
+        mbar_init(&ctl->idx_full[r], 1);
+        mbar_init(&ctl->idx_empty[r], kIdxReaders);
+      }
+    }
     ctl->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -1181,15 +1324,15 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100(const __grid_constan
 
   if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-    softmax_role<D, kOcc, kDense>(p, ctl, inv_l_sm, tmem, sP, warp >> 2, w);
+    softmax_role<D, kOcc, kDense, kClaim>(p, ctl, inv_l_sm, tmem, sP, warp >> 2, w);
   } else if (warp < 12) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
-    epilogue_role<D, kOcc>(p, ctl, inv_l_sm, tmem, w);
+    epilogue_role<D, kOcc, kClaim>(p, ctl, inv_l_sm, tmem, w);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
-    if (warp == kWarpMma && lane == 0) qk_role<D, kOcc>(p, ctl, tmem, sQ, sKV, w);
-    if (warp == kWarpPv && lane == 0) pv_role<D, kOcc>(p, ctl, tmem, sP, sKV, w);
-    if (warp == kWarpLoad && lane == 0) load_role<D, kOcc>(p, ctl, sQ, sKV, w);
+    if (warp == kWarpMma && lane == 0) qk_role<D, kOcc, kClaim>(p, ctl, tmem, sQ, sKV, w);
+    if (warp == kWarpPv && lane == 0) pv_role<D, kOcc, kClaim>(p, ctl, tmem, sP, sKV, w);
+    if (warp == kWarpLoad && lane == 0) load_role<D, kOcc, kClaim>(p, ctl, sQ, sKV, w);
   }
   __syncwarp();
   tc_fence_before();
@@ -1199,6 +1342,17 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100(const __grid_constan
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(C::kTmemCols)
                  : "memory");
+  }
+  if constexpr (kClaim) {
+    // Every claim of this CTA has returned (its TMA thread has left its
+    // list): the last CTA out leaves the counters at 0 for the next launch.
+    if (threadIdx.x == 0) {
+      __threadfence();
+      if (atomicAdd(p.claim_done, 1u) == gridDim.x - 1) {
+        atomicExch(p.claim, 0u);
+        atomicExch(p.claim_done, 0u);
+      }
+    }
   }
 }
 
@@ -1239,10 +1393,10 @@ bool encode_operand_map(CUtensorMap* tm, const void* base, int64_t D, int64_t S,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool kOcc, bool kDense>
+template <int D, bool kOcc, bool kDense, bool kClaim = false>
 static cudaError_t launch_d(const FwdParams& p, int grid, cudaStream_t stream, const char** why) {
   using C = dev::Cfg<D>;
-  auto kern = dev::fa_fwd_sm100<D, kOcc, kDense>;
+  auto kern = dev::fa_fwd_sm100<D, kOcc, kDense, kClaim>;
   static bool configured = false;
   static bool regs_ok = false;
   if (!configured) {
@@ -1267,18 +1421,23 @@ static cudaError_t launch_d(const FwdParams& p, int grid, cudaStream_t stream, c
 
 cudaError_t launch_fwd(int D, const FwdParams& p, int grid, cudaStream_t stream,
                        const char** why) {
-  // Three instances per head dim: ranges beside the items with and without
-  // the dense-mask extras, and ranges from the closed form (no item_tr).
+  // Four instances per head dim: ranges beside the items with the
+  // dense-mask extras, without them (fixed snake or claimed work), and
+  // ranges from the closed form (no item_tr). Only the claiming instance
+  // reads p.claim.
   const bool occ = p.item_tr != nullptr;
   const bool dense = occ && p.mask != nullptr && p.m_si > 0;
+  const bool claim = occ && !dense && p.claim != nullptr;
   if (D == 128)
-    return dense ? launch_d<128, true, true>(p, grid, stream, why)
-                 : occ ? launch_d<128, true, false>(p, grid, stream, why)
-                       : launch_d<128, false, false>(p, grid, stream, why);
+    return dense   ? launch_d<128, true, true>(p, grid, stream, why)
+           : claim ? launch_d<128, true, false, true>(p, grid, stream, why)
+           : occ   ? launch_d<128, true, false>(p, grid, stream, why)
+                   : launch_d<128, false, false>(p, grid, stream, why);
   if (D == 64)
-    return dense ? launch_d<64, true, true>(p, grid, stream, why)
-                 : occ ? launch_d<64, true, false>(p, grid, stream, why)
-                       : launch_d<64, false, false>(p, grid, stream, why);
+    return dense   ? launch_d<64, true, true>(p, grid, stream, why)
+           : claim ? launch_d<64, true, false, true>(p, grid, stream, why)
+           : occ   ? launch_d<64, true, false>(p, grid, stream, why)
+                   : launch_d<64, false, false>(p, grid, stream, why);
   if (why) *why = "unsupported head dim";
   return cudaErrorInvalidValue;
 }

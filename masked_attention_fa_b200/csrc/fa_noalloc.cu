@@ -12,7 +12,7 @@
 //
 // Limits and sharing:
 //   - The array holds kNoAllocScratchBytes (1 MiB): a 256-byte header (error
-//     word), the per-sequence records (32 bytes per sequence, rounded up to
+//     word and the kernel's two work-claim counters), the per-sequence records (32 bytes per sequence, rounded up to
 //     256 bytes) and the work list (16 bytes per (sequence, head, block of
 //     256 query rows)). Larger problems are rejected with FA_ERR_UNSUPPORTED
 //     before any device work.
@@ -282,6 +282,12 @@ extern "C" fa_status_t fa_fwd_noalloc(const fa_desc_t* desc, const void* q, cons
                           cudaMemcpyHostToDevice, stream);
       if (e != cudaSuccess) return cuda_err(e, "cudaMemcpyAsync(item ranges)");
       p.item_tr = reinterpret_cast<const TileRange*>(dscr + tr_off);
+      // Claimed work as in fa_fwd; the counters sit in the header, which
+      // was zeroed above.
+      if (n >= (size_t)kClaimMinItemsPerCta * (size_t)slot->num_sms && n < 0x7fff0000u) {
+        p.claim = reinterpret_cast<unsigned int*>(dscr + 128);
+        p.claim_done = reinterpret_cast<unsigned int*>(dscr + 192);
+      }
     }
   }
   if (has_mask && n > 0) {
