@@ -338,3 +338,13 @@ def test_paged_entry_point_validates_before_device_work():
     finally:
         fa.fa_destroy(tnd)
         fa.fa_destroy(bsnd)
+
+
+def test_claim_threshold_matches_the_library():
+    """The binding's CLAIM_MIN_ITEMS_PER_CTA (used to name the kernel instance a
+    call runs) is the library's kClaimMinItemsPerCta."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    with open(os.path.join(root, "masked_attention_fa_b200", "csrc", "fa_kernel.h")) as f:
+        m = re.search(r"constexpr int kClaimMinItemsPerCta = (\d+);", f.read())
+    assert m is not None
+    assert int(m.group(1)) == fa.CLAIM_MIN_ITEMS_PER_CTA
