@@ -342,6 +342,21 @@ fa_status_t fa_plan_stats(const fa_desc_t* desc, const int64_t* prefix,
                           const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
                           int32_t has_mask, int64_t* out);
 
+/*
+ * fa_plan_items — the work list of a closed-form call (no attenMask) in the
+ * order the kernel takes it: longest first by the cost key 8 x (the longer
+ * sub-tile's key tiles) + (the shorter's), ties in (sequence, block, head)
+ * order, so items without a key tile come last. Item m is out[4m .. 4m+3] =
+ * (sequence b, head h, block of 256 query rows, cost key). out: host
+ * int32[4 * capacity], may be NULL when capacity is 0. *n_items receives the
+ * list's length also when it exceeds capacity (then FA_ERR_SHAPE and out is
+ * not written). Host only; dense-mask calls rebuild their list on the device
+ * from the mask.
+ */
+fa_status_t fa_plan_items(const fa_desc_t* desc, const int64_t* prefix,
+                          const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
+                          int64_t capacity, int32_t* out, int64_t* n_items);
+
 /* ---------------- query split across devices (host only) ---------------- */
 
 /* One part of a query split: its own problem and where it sits in the

@@ -99,6 +99,9 @@ def load_library():
     lib.fa_tile_class.restype = ctypes.c_int32
     lib.fa_plan_stats.argtypes = [dp, i64p, i64p, i64p, ctypes.c_int32, i64p]
     lib.fa_plan_stats.restype = st
+    lib.fa_plan_items.argtypes = [dp, i64p, i64p, i64p, ctypes.c_int64,
+                                  ctypes.POINTER(ctypes.c_int32), i64p]
+    lib.fa_plan_items.restype = st
     lib.fa_fwd_noalloc.argtypes = [dp, P, P, P, P, i64p, i64p, i64p, P, P, P]
     lib.fa_fwd_noalloc.restype = st
     lib.fa_fwd_paged.argtypes = [P, P, P, P, P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
@@ -117,7 +120,8 @@ def load_library():
 
 EXPORTED = ("fa_create", "fa_fwd", "fa_sync_status", "fa_destroy", "fa_last_error",
             "fa_version", "fa_validate", "fa_visible_pairs", "fa_tile_class", "fa_plan_stats",
-            "fa_fwd_noalloc", "fa_split_queries", "fa_mask_occupancy", "fa_fwd_with_ranges", "fa_fwd_paged")
+            "fa_plan_items", "fa_fwd_noalloc", "fa_split_queries", "fa_mask_occupancy",
+            "fa_fwd_with_ranges", "fa_fwd_paged")
 
 
 def _check(status):
@@ -189,6 +193,23 @@ def fa_tile_class(desc, b, qt, kt, prefix=None, actual_seq_qlen=None, actual_seq
     a = _Arrays(prefix, actual_seq_qlen, actual_seq_kvlen)
     return int(load_library().fa_tile_class(ctypes.byref(desc), *a.ptrs(), int(bool(has_mask)),
                                              int(b), int(qt), int(kt)))
+
+
+def fa_plan_items(desc, prefix=None, actual_seq_qlen=None, actual_seq_kvlen=None):
+    """The closed-form work list in the kernel's order: int32 array [n, 4] of
+    (sequence, head, 256-row block, cost key)."""
+    import numpy as np
+    a = _Arrays(prefix, actual_seq_qlen, actual_seq_kvlen)
+    n = ctypes.c_int64(0)
+    lib = load_library()
+    st = lib.fa_plan_items(ctypes.byref(desc), *a.ptrs(), 0, None, ctypes.byref(n))
+    if n.value == 0:
+        _check(st)
+        return np.zeros((0, 4), dtype=np.int32)
+    out = np.zeros((n.value, 4), dtype=np.int32)
+    _check(lib.fa_plan_items(ctypes.byref(desc), *a.ptrs(), n.value,
+                             out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), ctypes.byref(n)))
+    return out
 
 
 def fa_plan_stats(desc, prefix=None, actual_seq_qlen=None, actual_seq_kvlen=None,

@@ -601,4 +601,28 @@ fa_status_t fa_plan_stats(const fa_desc_t* desc, const int64_t* prefix,
   return FA_OK;
 }
 
+fa_status_t fa_plan_items(const fa_desc_t* desc, const int64_t* prefix,
+                          const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
+                          int64_t capacity, int32_t* out, int64_t* n_items) {
+  clear_error();
+  if (!n_items) return fail(FA_ERR_NULLPTR, "n_items is NULL");
+  if (capacity < 0) return fail(FA_ERR_PARAM_INVALID, "capacity %lld < 0", (long long)capacity);
+  if (capacity > 0 && !out) return fail(FA_ERR_NULLPTR, "out is NULL");
+  fa_status_t st = validate_call(desc, prefix, actual_seq_qlen, actual_seq_kvlen, 0);
+  if (st != FA_OK) return st;
+  auto recs = decode_geometry(desc, prefix, actual_seq_qlen, actual_seq_kvlen, 0);
+  auto items = build_items(desc, recs);
+  *n_items = (int64_t)items.size();
+  if ((int64_t)items.size() > capacity)
+    return fail(FA_ERR_SHAPE, "the work list has %zu items, capacity %lld", items.size(),
+                (long long)capacity);
+  for (size_t m = 0; m < items.size(); ++m) {
+    out[4 * m] = items[m].b;
+    out[4 * m + 1] = items[m].h;
+    out[4 * m + 2] = items[m].qblk;
+    out[4 * m + 3] = items[m].cost;
+  }
+  return FA_OK;
+}
+
 }  // extern "C"

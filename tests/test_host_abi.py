@@ -348,3 +348,73 @@ def test_claim_threshold_matches_the_library():
         m = re.search(r"constexpr int kClaimMinItemsPerCta = (\d+);", f.read())
     assert m is not None
     assert int(m.group(1)) == fa.CLAIM_MIN_ITEMS_PER_CTA
+
+
+# Work lists of closed-form calls, checked against the oracle's own tile
+# ranges (from its visibility definition): every (sequence, head, block of
+# 256 query rows) with a query row appears once, the cost keys are
+# 8 x (the longer sub-tile's key tiles) + (the shorter's) and never increase
+# along the list, so items without a key tile come last (the claiming kernel
+# relies on that), and equal keys keep (sequence, block, head) order.
+PLAN_CASES = [
+    dict(layout="BNSD", B=2, N=3, Sq=700, Skv=900, D=64, sparse_mode=2),
+    dict(layout="BNSD", B=1, N=2, Sq=1000, Skv=600, D=64, sparse_mode=3),
+    dict(layout="BSND", B=2, N=2, Sq=800, Skv=2000, D=128, sparse_mode=4, pre_tokens=300,
+         next_tokens=0),
+    dict(layout="BNSD", B=3, N=2, Sq=900, Skv=900, D=64, sparse_mode=5, prefix=[0, 200, 900]),
+    dict(layout="BNSD", B=1, N=2, Sq=600, Skv=700, D=64, sparse_mode=0),
+    dict(layout="TND", B=6, N=2, Sq=0, Skv=0, D=64, sparse_mode=3,
+         qlen=[300, 0, 129, 700, 5, 256], kvlen=[400, 50, 0, 900, 5, 1]),
+    dict(layout="TND", B=2, N=2, Sq=5, Skv=9, D=64, sparse_mode=7, pre_tokens=6, next_tokens=-2,
+         qlen=[3, 2], kvlen=[3, 6]),
+    dict(layout="TND", B=3, N=2, Sq=12, Skv=13, D=64, sparse_mode=8, pre_tokens=4, next_tokens=1,
+         qlen=[3, 5, 4], kvlen=[4, 5, 4]),
+]
+
+
+@pytest.mark.parametrize("case", range(len(PLAN_CASES)))
+def test_work_list_order_and_keys_match_the_oracle_ranges(case):
+    c = dict(PLAN_CASES[case])
+    qlen, kvlen = c.pop("qlen", None), c.pop("kvlen", None)
+    prefix = c.pop("prefix", None)
+    cu_q = cu_kv = None
+    if qlen is not None:
+        cu_q, cu_kv = np.cumsum(qlen).tolist(), np.cumsum(kvlen).tolist()
+        c["Sq"], c["Skv"] = cu_q[-1], cu_kv[-1]
+    desc = fa.make_desc(**c)
+    items = fa.fa_plan_items(desc, prefix=prefix, actual_seq_qlen=cu_q, actual_seq_kvlen=cu_kv)
+    pb = Problem(**c, prefix=prefix, actual_seq_qlen=cu_q, actual_seq_kvlen=cu_kv)
+    expected = {}
+    for b in range(c["B"]):
+        sq = pb.seq(b)[2]
+        if sq <= 0:
+            continue
+        r = oracle.tile_ranges(oracle.tile_classes(pb, b))
+        tiles = [int(r[qt, 1] - r[qt, 0]) if qt < len(r) else 0 for qt in range(len(r) + 1)]
+        for qb in range((sq + 255) // 256):
+            t0, t1 = tiles[2 * qb], tiles[2 * qb + 1]
+            for h in range(c["N"]):
+                expected[(b, h, qb)] = 8 * max(t0, t1) + min(t0, t1)
+    got = {(int(b), int(h), int(qb)): int(key) for b, h, qb, key in items}
+    assert len(got) == len(items), "an item appears twice"
+    assert got == expected
+    keys = items[:, 3]
+    assert np.all(keys[:-1] >= keys[1:]), "keys must not increase along the list"
+    for m in range(len(items) - 1):
+        if keys[m] == keys[m + 1]:
+            a, z = items[m], items[m + 1]
+            assert (a[0], a[2], a[1]) < (z[0], z[2], z[1]), "ties keep (sequence, block, head) order"
+
+
+def test_plan_items_reports_its_length_and_rejects_a_short_buffer():
+    import ctypes
+    desc = fa.make_desc("BNSD", 1, 2, 600, 600, 64, 2)
+    lib = fa.load_library()
+    n = ctypes.c_int64(-1)
+    buf = (ctypes.c_int32 * 8)()
+    st = lib.fa_plan_items(ctypes.byref(desc), None, None, None, 2, buf, ctypes.byref(n))
+    assert fa.STATUS[st] == "FA_ERR_SHAPE" and n.value == 6   # 3 blocks x 2 heads
+    st = lib.fa_plan_items(ctypes.byref(desc), None, None, None, 0, None, None)
+    assert fa.STATUS[st] == "FA_ERR_NULLPTR"
+    st = lib.fa_plan_items(ctypes.byref(desc), None, None, None, 4, None, ctypes.byref(n))
+    assert fa.STATUS[st] == "FA_ERR_NULLPTR"
