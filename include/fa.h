@@ -175,7 +175,7 @@ int32_t fa_version(void);
  * allocate memory (for example code running inside a framework that owns
  * every device allocation through its own pool, a real-time loop that must
  * not allocate after start-up, or a plugin called from another library's
- * memory callbacks). The paper has no counterpart of this entry point.
+ * memory callbacks). The pages have no counterpart of this entry point.
  *
  * No handle: the descriptor and all arrays are passed on every call, with
  * the meaning, layout and validation of fa_create + fa_fwd. The work list
@@ -191,8 +191,13 @@ int32_t fa_version(void);
  * and 128 x 128 tile) behind the work list when they fit; when they do not,
  * the call runs without the pre-pass (every tile of the band with the
  * element mask) and gives the same result.
+ * A closed-form call puts each item's two key-tile ranges behind the list
+ * when they fit, and then, with at least 8 items per SM, claims its items
+ * through two counters in the array's 256-byte header, cleared with the
+ * error word (see fa_fwd, work distribution).
  * Sharing: every call shares the array and leaves its work list there; the
- * error word is cleared at the start of each call. Calls whose kernels
+ * header (error word and claim counters) is cleared at the start of each
+ * call. Calls whose kernels
  * overlap on the GPU race on the array: order them on one stream. Host calls
  * are serialised internally.
  * Set-up: the first call on each device looks up the array's device address
