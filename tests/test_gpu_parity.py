@@ -94,51 +94,125 @@ def test_varlen_tnd_matches_oracle(case, D):
     check_against_oracle(kw, inp, prefix=prefix, cu_q=cu_q, cu_kv=cu_k)
 
 
+def _probe_mask(kind, B, N, Sq, Skv, seed, dead_rows=()):
+    """A Bernoulli(0.25) uint8 mask of the given kind, with rows in
+    `dead_rows` hidden entirely (rows that see no key)."""
+    shape = {"SS": (Sq, Skv), "B1SS": (B, 1, Sq, Skv), "BNSS": (B, N, Sq, Skv)}[kind]
+    g = torch.Generator().manual_seed(seed)
+    m = (torch.rand(shape, generator=g) < 0.25).to(torch.uint8)
+    for r in dead_rows:
+        m[..., r, :] = 1
+    return m
+
+
+# (layout, mode, extra kwargs, B, N, Sq or lens_q, Skv or lens_kv, prefix, mask spec)
 PROBE_CASES = [
-    ("BNSD", 2, {}, 200, 300, None),
-    ("BNSD", 3, {}, 300, 200, None),
-    ("BSND", 4, dict(pre_tokens=50, next_tokens=-10), 300, 330, None),
-    ("BNSD", 5, {}, 260, 260, [70]),
-    ("BNSD", 0, dict(pre_tokens=40, next_tokens=3, mask_kind="SS"), 200, 260, None),
+    ("BNSD", 2, {}, 1, 1, 200, 300, None, None),
+    ("BNSD", 3, {}, 1, 1, 300, 200, None, None),
+    ("BSND", 4, dict(pre_tokens=50, next_tokens=-10), 1, 1, 300, 330, None, None),
+    # the right-down band across many key tiles (each sub-tile has two
+    # boundary tiles and several full ones)
+    ("BSND", 4, dict(pre_tokens=300, next_tokens=0), 1, 2, 256, 1024, None, None),
+    ("BNSD", 5, {}, 1, 1, 260, 260, [70], None),
+    ("BNSD", 5, {}, 2, 1, 200, 333, [0, 333], None),
+    ("BNSD", 6, {}, 1, 1, 300, 520, [130], None),
+    ("BNSD", 0, dict(pre_tokens=40, next_tokens=3, mask_kind="SS"), 1, 1, 200, 260, None,
+     ("SS", ())),
+    ("BSND", 0, dict(pre_tokens=150, next_tokens=-40, mask_kind="B1SS"), 2, 2, 260, 300, None,
+     ("B1SS", (5, 131))),
+    ("BNSD", 1, dict(mask_kind="SS"), 1, 1, 200, 300, None, ("SS", (0, 77, 199))),
+    ("BNSD", 1, dict(mask_kind="BNSS"), 2, 2, 150, 260, None, ("BNSS", (3, 128, 149))),
+    ("BSND", 1, dict(mask_kind="B1SS"), 2, 2, 129, 385, None, ("B1SS", (128,))),
+    # varlen: the two worked split examples, unsplit and per card
+    ("TND", 3, {}, 4, 2, [3, 4, 5, 4], [3, 6, 5, 4], None, None),
+    ("TND", 7, dict(pre_tokens=6, next_tokens=-2), 2, 2, [3, 2], [3, 6], None, None),
+    ("TND", 3, {}, 3, 2, [2, 5, 4], [6, 5, 4], None, None),
+    ("TND", 2, {}, 4, 2, [3, 5, 5, 4], [3, 4, 5, 4], None, None),
+    ("TND", 2, {}, 2, 2, [3, 2], [3, 4], None, None),
+    ("TND", 8, dict(pre_tokens=4, next_tokens=1), 3, 2, [3, 5, 4], [4, 5, 4], None, None),
+    # varlen with empty sequences (a trailing one, one in the middle)
+    ("TND", 3, {}, 4, 2, [130, 0, 257, 0], [140, 3, 300, 0], None, None),
+    # modes 7 and 8 with a band sequence spanning several key tiles
+    ("TND", 7, dict(pre_tokens=1000, next_tokens=-100), 3, 2, [100, 0, 700], [150, 3, 1000],
+     None, None),
+    ("TND", 8, dict(pre_tokens=950, next_tokens=-50), 3, 2, [0, 600, 300], [3, 900, 350], None,
+     None),
+    ("TND", 4, dict(pre_tokens=60, next_tokens=10), 2, 1, [200, 129], [260, 400], None, None),
+    ("TND", 5, {}, 3, 1, [150, 1, 257], [150, 2, 300], [17, 0, 300], None),
 ]
+
+
+def _probe_case(case):
+    layout, mode, extra, B, N, sq, skv, prefix, mspec = PROBE_CASES[case]
+    cu_q = cu_kv = None
+    if layout == "TND":
+        cu_q, cu_kv = np.cumsum(sq).tolist(), np.cumsum(skv).tolist()
+        sq, skv = cu_q[-1], cu_kv[-1]
+    mask = None
+    if mspec is not None:
+        mask = _probe_mask(mspec[0], B, N, sq, skv, seed=7 + case, dead_rows=mspec[1])
+    return _kw(layout, B, N, sq, skv, None, mode, **extra), mask, prefix, cu_q, cu_kv
 
 
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("case", range(len(PROBE_CASES)))
 def test_visibility_probe_is_exact(case, D):
-    """Q = K = 0 and V = the identity on key block c: O[i, j - cD] != 0
-    exactly when key j is visible to row i, and lse_i = ln |vis(i)|."""
-    layout, mode, extra, Sq, Skv, prefix = PROBE_CASES[case]
-    extra = dict(extra)
-    B, N = 1, 1
-    kw = _kw(layout, B, N, Sq, Skv, D, mode, **extra)
-    mask = None
-    if kw.get("mask_kind"):
-        g = torch.Generator().manual_seed(7)
-        mask = (torch.rand(Sq, Skv, generator=g) < 0.25).to(torch.uint8)
-    pb = problem_of(kw, mask, prefix)
-    vis = oracle.mask_matrix(pb, 0)
-    shape_q = (B, N, Sq, D) if layout == "BNSD" else (B, Sq, N, D)
-    shape_kv = (B, N, Skv, D) if layout == "BNSD" else (B, Skv, N, D)
+    """Q = K = 0 and, for key block c of every sequence, V = the identity on
+    that block (V[j, j - cD] = 1): then O[i, j - cD] != 0 exactly when key j
+    is visible to row i (every visible key gets the same weight 1/|vis(i)|,
+    a power-of-two fraction or a bf16 value well above 0, every hidden key
+    exactly 0), for every sequence and head; and lse_i = ln |vis(i)|, -inf
+    for a row that sees no key. Compared with the oracle's visibility matrix
+    with no tolerance."""
+    kw, mask, prefix, cu_q, cu_kv = _probe_case(case)
+    kw["D"] = D
+    layout, B, N, Sq, Skv = kw["layout"], kw["B"], kw["N"], kw["Sq"], kw["Skv"]
+    pb = problem_of(kw, mask, prefix, cu_q, cu_kv)
+    seqs = [pb.seq(b) for b in range(B)]
+    shape_q = pb.q_shape()
+    shape_kv = pb.kv_shape()
     q = torch.zeros(shape_q, dtype=torch.bfloat16)
     k = torch.zeros(shape_kv, dtype=torch.bfloat16)
-    seen = np.zeros((Sq, Skv), dtype=bool)
-    for c in range((Skv + D - 1) // D):
+    seen = {(b, h): np.zeros((s[2], s[3]), dtype=bool) for b, s in enumerate(seqs)
+            for h in range(N)}
+    lse_all = None
+    n_blocks = max((s[3] + D - 1) // D for s in seqs) if seqs else 0
+    for c in range(max(n_blocks, 1)):
         v = torch.zeros(shape_kv, dtype=torch.bfloat16)
-        for j in range(c * D, min(Skv, (c + 1) * D)):
-            if layout == "BNSD":
-                v[0, 0, j, j - c * D] = 1
-            else:
-                v[0, j, 0, j - c * D] = 1
-        o, lse = run_cuda(kw, q, k, v, mask, prefix)
-        o2 = o[0, 0] if layout == "BNSD" else o[0, :, 0]
-        w = min(Skv, (c + 1) * D) - c * D
-        seen[:, c * D:c * D + w] = o2[:, :w] != 0
-    assert np.array_equal(seen, vis.astype(bool))
-    cnt = vis.sum(1)
-    lse_row = lse[0, 0]
-    assert np.all(np.isneginf(lse_row[cnt == 0]))
-    np.testing.assert_allclose(lse_row[cnt > 0], np.log(cnt[cnt > 0]), rtol=0, atol=TOL_LSE)
+        for b, (_, k0, _, skv_b) in enumerate(seqs):
+            if skv_b <= c * D:
+                continue
+            jj = torch.arange(c * D, min(skv_b, (c + 1) * D))
+            for h in range(N):
+                if layout == "BNSD":
+                    v[b, h, jj, jj - c * D] = 1
+                elif layout == "BSND":
+                    v[b, jj, h, jj - c * D] = 1
+                else:
+                    v[k0 + jj, h, jj - c * D] = 1
+        o, lse = run_cuda(kw, q, k, v, mask, prefix, cu_q, cu_kv)
+        lse_all = lse
+        for b, (q0, _, sq_b, skv_b) in enumerate(seqs):
+            w = min(skv_b, (c + 1) * D) - c * D
+            if w <= 0 or sq_b == 0:
+                continue
+            for h in range(N):
+                if layout == "BNSD":
+                    ob = o[b, h]
+                elif layout == "BSND":
+                    ob = o[b, :, h]
+                else:
+                    ob = o[q0:q0 + sq_b, h]
+                seen[(b, h)][:, c * D:c * D + w] = ob[:, :w] != 0
+    for b, (q0, _, sq_b, skv_b) in enumerate(seqs):
+        for h in range(N):
+            vis = oracle.mask_matrix(pb, b, h).astype(bool)
+            assert np.array_equal(seen[(b, h)], vis), (b, h)
+            cnt = vis.sum(1)
+            lrow = lse_all[h, q0:q0 + sq_b] if layout == "TND" else lse_all[b, h]
+            assert np.all(np.isneginf(lrow[cnt == 0])), (b, h)
+            np.testing.assert_allclose(lrow[cnt > 0], np.log(cnt[cnt > 0]), rtol=0,
+                                       atol=TOL_LSE)
 
 
 @pytest.mark.parametrize("D", [64, 128])

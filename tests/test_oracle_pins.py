@@ -637,3 +637,54 @@ def test_paged_decode_row_is_sdpa_over_the_gathered_keys():
         np.testing.assert_allclose(o[b], ref, rtol=0, atol=1e-12)
         s = pb.scale * np.einsum("hd,nhd->hn", q[b], kb)
         np.testing.assert_allclose(l[:, b], np.log(np.exp(s).sum(1)), rtol=0, atol=1e-12)
+
+
+def _runs_of_full(row):
+    """Every maximal run of class-2 blocks as (start, end)."""
+    runs, k = [], 0
+    while k < len(row):
+        if row[k] == 2:
+            e = k
+            while e < len(row) and row[e] == 2:
+                e += 1
+            runs.append((k, e))
+            k = e
+        else:
+            k += 1
+    return runs
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_tile_ranges_properties_on_random_class_rows(seed):
+    """Properties any correct block range must have, on random class rows:
+    [lo, hi) holds every non-empty block and starts and ends on one; nothing
+    outside it is non-empty; [full_lo, full_hi) holds only full blocks and is
+    a maximal run that no other run of full blocks is longer than (on ties no
+    earlier run is as long); with no full block it is the empty run at lo.
+    These do not depend on the loop the oracle uses to find them."""
+    rng = np.random.default_rng(seed)
+    n_qt, n_kt = 40, int(rng.integers(1, 30))
+    p = rng.dirichlet([1.0, 1.0, 1.0])
+    cls = rng.choice(3, size=(n_qt, n_kt), p=p).astype(np.uint8)
+    cls[0] = 0                        # a query block without a visible pair
+    cls[1] = 2                        # one that is full end to end
+    got = oracle.tile_ranges(cls)
+    for qt in range(n_qt):
+        row = cls[qt]
+        lo, hi, flo, fhi = (int(x) for x in got[qt])
+        nz = np.flatnonzero(row)
+        if nz.size == 0:
+            assert (lo, hi, flo, fhi) == (0, 0, 0, 0)
+            continue
+        assert lo == nz[0] and hi == nz[-1] + 1          # tight cover of the non-empty blocks
+        assert not row[:lo].any() and not row[hi:].any()
+        runs = _runs_of_full(row)
+        if not runs:
+            assert (flo, fhi) == (lo, lo)
+            continue
+        assert lo <= flo < fhi <= hi
+        assert np.all(row[flo:fhi] == 2)
+        assert (flo, fhi) in runs                         # a maximal run, not part of one
+        longest = max(e - s for s, e in runs)
+        assert fhi - flo == longest
+        assert all(s >= flo for s, e in runs if e - s == longest)
