@@ -6,8 +6,10 @@ Prints ONE JSON line (rank 0). A step is one fa_fwd over the whole workload
 (every KV tile of every (sequence, head, query block)). The metric counts
 only visible (i, j) pairs: TFLOP/s = 4 * D * pairs / time.
 
-Default workload: B=2, N=16, Sq=Skv=4096, D=128, BNSD, sparseMode 2
-(leftUpCausal), bf16 N(0,1) inputs from seed 2. With --gpus N > 1 (under
+Default workload: prefix_8k, B=4, N=16, Sq=Skv=8192, D=128, BNSD, sparseMode 5
+(rightDownCausal plus the per-batch prefix [512, 1024, 2048, 4096]), bf16
+N(0,1) inputs from seed 5: the largest of the causal, band and prefix
+scenarios (1.19 TFLOP of visible work per call). With --gpus N > 1 (under
 torchrun) every rank runs its own independent copy of the workload (the
 work shards by (batch, head, query block) with no exchange), so the value
 is the total over ranks divided by the slowest rank's time (weak scaling).
@@ -32,7 +34,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-DEFAULT_WORKLOAD = "leftup_causal_4k"
+DEFAULT_WORKLOAD = "prefix_8k"
 METRIC = "masked-attention fwd TFLOP/s (visible pairs) and % of B200 BF16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -301,6 +303,38 @@ def cpu_baseline_sample(w, inputs, seconds):
     return tflops, oracle.num_threads(), desc
 
 
+def bench_config(w, pairs, world):
+    """The `config` object of the JSON line, the same for both arms."""
+    paged = w.block_size is not None
+    return {"workload": w.name, "layout": w.layout, "B": w.B, "N": w.N, "Sq": w.Sq,
+            "Skv": w.Skv, "D": w.D, "sparse_mode": w.sparse_mode, "visible_pairs": int(pairs),
+            "per_rank": "independent copy",
+            "l2": "cold: a 256 MiB buffer is written between timed GPU steps",
+            **({"block_size": w.block_size, "kv_cache": "paged, resident"} if paged else {}),
+            "parallelism": f"replicas x{world}"}
+
+
+def oracle_visible_pairs(w, mask_host=None):
+    """Visible pairs of the workload counted from the oracle's explicit
+    visibility matrices (one per sequence; per head only for a BNSS mask)."""
+    import numpy as np
+    import oracle
+    from oracle import Problem
+    kw = dict(layout=w.layout, B=w.B, N=w.N, Sq=w.Sq, Skv=w.Skv, D=w.D,
+              sparse_mode=w.sparse_mode, pre_tokens=w.pre_tokens, next_tokens=w.next_tokens,
+              scale=w.scale, prefix=w.prefix, actual_seq_qlen=w.actual_seq_qlen,
+              actual_seq_kvlen=w.actual_seq_kvlen)
+    if mask_host is not None:
+        kw.update(mask=mask_host.numpy(), mask_kind=w.mask_kind)
+    pb = Problem(**kw)
+    total = 0
+    for b in range(w.B):
+        heads = range(w.N) if w.mask_kind == "BNSS" else [0]
+        per = sum(int(oracle.mask_matrix(pb, b, h).sum(dtype=np.int64)) for h in heads)
+        total += per if w.mask_kind == "BNSS" else per * w.N
+    return total
+
+
 def run_reference(args):
     """The oracle on the host cores, as the reference arm."""
     rank = int(os.environ.get("RANK", "0"))
@@ -324,12 +358,15 @@ def run_reference(args):
         if s >= args.warmup:
             vals.append(tf)
     value = statistics.median(vals)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if w.block_size is not None:
+        pairs = sum(sq * skv for sq, skv in w.seq_lens()) * w.N  # decode rows see every key
+    else:
+        pairs = oracle_visible_pairs(w, inputs.get("mask"))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": w.name, "layout": w.layout, "B": w.B,
-                                            "N": w.N, "Sq": w.Sq, "Skv": w.Skv, "D": w.D,
-                                            "sparse_mode": w.sparse_mode},
+            "data": "synthetic", "config": bench_config(w, pairs, world),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -563,13 +600,7 @@ def main():
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": w.name, "layout": w.layout, "B": w.B, "N": w.N,
-                           "Sq": w.Sq, "Skv": w.Skv, "D": w.D, "sparse_mode": w.sparse_mode,
-                           "visible_pairs": pairs, "per_rank": "independent copy",
-                           "l2": "256 MiB buffer written between timed steps (cold L2)",
-                           **({"block_size": w.block_size, "kv_cache": "paged, resident"}
-                              if paged else {}),
-                           "parallelism": f"replicas x{world}"},
+                "config": bench_config(w, pairs, world),
                 "frac_of_peak": value / world / peak,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": args.steps * (4 if dense else (2 if paged else 1)),

@@ -203,13 +203,35 @@ int32_t fa_version(void);
  * Set-up: the first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) and the device's attributes with that device
  * current; make that first call before any stream capture begins.
- * A device-side wait that gives up leaves the outputs undefined and is not
- * reported by this entry point.
+ * Graphs: calls cannot be captured into a CUDA graph. Each call uploads its
+ * work list from one static host buffer that the next call overwrites, so a
+ * replay would read another call's list; a call on a capturing stream
+ * returns FA_ERR_UNSUPPORTED and enqueues nothing.
+ * Device-side failures: a bounded wait in the kernel that gives up leaves
+ * the outputs undefined and sets an error word in the array's header, which
+ * fa_noalloc_sync_status reports. Each call clears the header first, so the
+ * word describes the most recent call.
  */
 fa_status_t fa_fwd_noalloc(const fa_desc_t* desc, const void* q, const void* k, const void* v,
                            const uint8_t* atten_mask, const int64_t* prefix,
                            const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
                            void* o, float* lse, void* cuda_stream);
+
+/*
+ * fa_noalloc_sync_status — the fa_sync_status of the allocation-free entry
+ * point (which has no handle to hold its status). The pages have no
+ * counterpart of it.
+ *
+ * Waits for `cuda_stream` (the stream of the last fa_fwd_noalloc call on
+ * the current device), then reads the error word in the fixed array's
+ * header: FA_OK, FA_ERR_TIMEOUT (a bounded wait in the kernel gave up; that
+ * call's O and lse are undefined) or FA_ERR_DEVICE. A non-zero word is
+ * cleared, with the rest of the header. Allocates nothing (the word is read
+ * into a static host variable). FA_OK when no call has run on the device.
+ * Errors: FA_ERR_CUDA if the synchronisation or the read fails (for example
+ * after a fault that ended the CUDA context).
+ */
+fa_status_t fa_noalloc_sync_status(void* cuda_stream);
 
 /*
  * fa_fwd_paged — forward of a TND handle with the keys and values read from

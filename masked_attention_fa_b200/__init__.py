@@ -104,6 +104,8 @@ def load_library():
     lib.fa_plan_items.restype = st
     lib.fa_fwd_noalloc.argtypes = [dp, P, P, P, P, i64p, i64p, i64p, P, P, P]
     lib.fa_fwd_noalloc.restype = st
+    lib.fa_noalloc_sync_status.argtypes = [P]
+    lib.fa_noalloc_sync_status.restype = st
     lib.fa_fwd_paged.argtypes = [P, P, P, P, P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                  i64p, i64p, i64p, P, P, P]
     lib.fa_fwd_paged.restype = st
@@ -121,7 +123,7 @@ def load_library():
 EXPORTED = ("fa_create", "fa_fwd", "fa_sync_status", "fa_destroy", "fa_last_error",
             "fa_version", "fa_validate", "fa_visible_pairs", "fa_tile_class", "fa_plan_stats",
             "fa_plan_items", "fa_fwd_noalloc", "fa_split_queries", "fa_mask_occupancy",
-            "fa_fwd_with_ranges", "fa_fwd_paged")
+            "fa_fwd_with_ranges", "fa_fwd_paged", "fa_noalloc_sync_status")
 
 
 def _check(status):
@@ -322,6 +324,22 @@ def fa_fwd_noalloc(desc, q, k, v, o, lse, atten_mask=None, prefix=None, actual_s
     _check(load_library().fa_fwd_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v),
                                          _ptr(atten_mask), *a.ptrs(), _ptr(o), _ptr(lse),
                                          ctypes.c_void_p(int(stream))))
+
+
+def fa_noalloc_sync_status(stream=None, raise_on_error=True):
+    """Wait for `stream` and read the error word of the allocation-free
+    path's fixed array (see include/fa.h); returns the status code, or
+    raises FaError for a non-OK status when raise_on_error."""
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    elif hasattr(stream, "cuda_stream"):
+        stream = stream.cuda_stream
+    lib = load_library()
+    st = lib.fa_noalloc_sync_status(ctypes.c_void_p(int(stream)))
+    if raise_on_error:
+        _check(st)
+    return st
 
 
 def fa_split_queries(desc, actual_seq_qlen, actual_seq_kvlen, n_parts, part, cuts=None):

@@ -608,8 +608,10 @@ fa_status_t fa_sync_status(fa_handle_t h) {
   e = cudaMemcpy(&word, h->d_ws, sizeof(word), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(error word)");
   if (word == 0) return FA_OK;
-  e = cudaMemset(h->d_ws, 0, sizeof(word));
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(error word)");
+  // Clear the whole header: the error word and, should an aborted launch
+  // have left them set, the claim counters.
+  e = cudaMemset(h->d_ws, 0, kHeaderBytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(header)");
   if (word & kErrTimeout)
     return fail(FA_ERR_TIMEOUT, "a device-side wait gave up (site %u); outputs are undefined",
                 (word >> kErrWhereShift) & 0xffu);

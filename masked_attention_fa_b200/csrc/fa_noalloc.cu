@@ -31,6 +31,14 @@
 //     array's device address with cudaGetSymbolAddress, reads the device's
 //     attributes and sets the kernel's shared-memory attribute). Make that
 //     first call before any stream capture begins.
+//   - Calls cannot be recorded into a CUDA graph: each call uploads its work
+//     list from one static host image that the next call overwrites, so a
+//     replayed copy would pair this call's outputs with another call's list.
+//     A call on a stream that is capturing returns FA_ERR_UNSUPPORTED before
+//     doing anything.
+//   - A device-side wait that gives up leaves an error word in the array's
+//     header; fa_noalloc_sync_status reads it (and clears the header). The
+//     next call clears it too, so check after each call that needs checking.
 //   - No cudaMalloc, cudaFree, pinned or host-heap allocation happens on the
 //     success path: the work list is built in a static host buffer, copied
 //     with cudaMemcpyAsync from pageable memory (the call returns once the
@@ -39,6 +47,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -73,6 +82,21 @@ struct DeviceSlot {
 DeviceSlot g_devices[kNoAllocMaxDevices];
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+// The test hooks the handle path reads at fa_create (a dropped first Q load
+// that makes a bounded wait run out, and a shorter wait limit), read here at
+// every call: reading the environment allocates nothing.
+bool env_flag(const char* name) {
+  const char* v = std::getenv(name);
+  return v != nullptr && v[0] != '\0' && v[0] != '0';
+}
+uint64_t wait_limit_ns() {
+  if (const char* t = std::getenv("FA_WAIT_TIMEOUT_MS")) {
+    const long long ms = std::atoll(t);
+    if (ms > 0) return (uint64_t)ms * 1000000ull;
+  }
+  return 2000000000ull;
+}
 
 fa_status_t cuda_err(cudaError_t e, const char* what) {
   return fail(FA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
@@ -154,6 +178,17 @@ extern "C" fa_status_t fa_fwd_noalloc(const fa_desc_t* desc, const void* q, cons
                 need, kNoAllocScratchBytes, (long long)desc->B, n_items);
   if (n_items == 0) return FA_OK;
 
+  // A graph replay of this call would re-read the static host image after
+  // later calls rewrote it: refuse capture outright.
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  cudaStreamCaptureStatus capturing = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(stream, &capturing);
+  if (e != cudaSuccess) return cuda_err(e, "cudaStreamIsCapturing");
+  if (capturing != cudaStreamCaptureStatusNone)
+    return fail(FA_ERR_UNSUPPORTED,
+                "fa_fwd_noalloc cannot be captured into a CUDA graph (its work list is uploaded "
+                "from a host buffer that later calls overwrite); call it outside capture");
+
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceSlot* slot = nullptr;
   st = device_slot(&slot);
@@ -228,9 +263,8 @@ extern "C" fa_status_t fa_fwd_noalloc(const fa_desc_t* desc, const void* q, cons
     return a.h < c.h;
   });
 
-  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   unsigned char* dscr = static_cast<unsigned char*>(slot->scratch);
-  cudaError_t e = cudaMemsetAsync(dscr, 0, kNoAllocHeaderBytes, stream);  // error word = 0
+  e = cudaMemsetAsync(dscr, 0, kNoAllocHeaderBytes, stream);  // error word = 0
   if (e != cudaSuccess) return cuda_err(e, "cudaMemsetAsync");
   e = cudaMemcpyAsync(dscr + kNoAllocHeaderBytes, g_host_image + kNoAllocHeaderBytes,
                       need - kNoAllocHeaderBytes, cudaMemcpyHostToDevice, stream);
@@ -332,8 +366,8 @@ extern "C" fa_status_t fa_fwd_noalloc(const fa_desc_t* desc, const void* q, cons
   p.n_items = (int32_t)n;
   p.tnd = tnd ? 1 : 0;
   p.scale_log2 = (float)(d->scale * 1.4426950408889634073599);
-  p.debug_flags = 0;
-  p.timeout_ns = 2000000000ull;
+  p.debug_flags = env_flag("FA_TEST_DROP_FIRST_Q") ? kDebugDropFirstQ : 0u;
+  p.timeout_ns = wait_limit_ns();
   const int grid = (int)std::min<size_t>(n, (size_t)slot->num_sms);
   const char* why = nullptr;
   e = launch_fwd((int)d->D, p, grid, stream, &why);
@@ -342,4 +376,30 @@ extern "C" fa_status_t fa_fwd_noalloc(const fa_desc_t* desc, const void* q, cons
     return cuda_err(e, "kernel launch");
   }
   return FA_OK;
+}
+
+extern "C" fa_status_t fa_noalloc_sync_status(void* cuda_stream) {
+  clear_error();
+  std::lock_guard<std::mutex> lock(g_mutex);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_err(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kNoAllocMaxDevices || !g_devices[dev].ready)
+    return FA_OK;  // no call has run on this device
+  e = cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) return cuda_err(e, "cudaStreamSynchronize");
+  // A 4-byte read into a static host word: no allocation.
+  static unsigned int word;
+  e = cudaMemcpy(&word, g_devices[dev].scratch, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_err(e, "cudaMemcpy(error word)");
+  if (word == 0) return FA_OK;
+  // Clear the whole header: the error word and, should an aborted launch
+  // have left them set, the claim counters.
+  e = cudaMemset(g_devices[dev].scratch, 0, kNoAllocHeaderBytes);
+  if (e != cudaSuccess) return cuda_err(e, "cudaMemset(header)");
+  if (word & kErrTimeout)
+    return fail(FA_ERR_TIMEOUT,
+                "a device-side wait gave up (site %u); the last call's outputs are undefined",
+                (word >> kErrWhereShift) & 0xffu);
+  return fail(FA_ERR_DEVICE, "device error word 0x%08x", word);
 }
