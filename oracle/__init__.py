@@ -24,6 +24,8 @@ _SRC = os.path.join(_HERE, "fa_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 LAYOUTS = {"BNSD": 0, "BSND": 1, "TND": 2}
+# ALiBi variants of the "压缩mask" page's alibi section.
+ALIBI = {None: 0, "right": 1, "sqrt": 2, "left": 3}
 MASK_KINDS = {None: 0, "SS": 1, "B1SS": 2, "BNSS": 3}
 
 
@@ -68,6 +70,9 @@ def _load():
         lib.oracle_visible.restype = ctypes.c_int
         lib.oracle_attn.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, P, P, P, P, P]
         lib.oracle_attn.restype = ctypes.c_int
+        lib.oracle_attn_alibi.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, ctypes.c_int32, P,
+                                          P, P, P, P, P]
+        lib.oracle_attn_alibi.restype = ctypes.c_int
         lib.oracle_attn_rows.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, P, P, P, i64, P, P, P]
         lib.oracle_attn_rows.restype = ctypes.c_int
         lib.oracle_mask.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, i64, i64, P]
@@ -212,16 +217,25 @@ def visible_count(pb: Problem) -> int:
     return int(_load().oracle_visible_count(ctypes.byref(d), pre, cq, ckv, m))
 
 
-def attention(pb: Problem, q, k, v):
-    """Full forward in fp64: returns (O in Q's layout, lse)."""
+def attention(pb: Problem, q, k, v, alibi=None, slopes=None):
+    """Full forward in fp64: returns (O in Q's layout, lse). With alibi in
+    ("right", "sqrt", "left") and slopes [N], each visible score gets
+    slopes[h] times that variant's bias added."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     assert q.shape == pb.q_shape() and k.shape == pb.kv_shape() and v.shape == pb.kv_shape()
     o = np.zeros(pb.q_shape(), dtype=np.float64)
     lse = np.full(pb.lse_shape(), -np.inf, dtype=np.float64)
     d = pb.desc()
     pre, cq, ckv, m = pb._ptrs()
-    err = _load().oracle_attn(ctypes.byref(d), pre, cq, ckv, m, q.ctypes.data, k.ctypes.data,
-                              v.ctypes.data, o.ctypes.data, lse.ctypes.data)
+    if alibi is None:
+        err = _load().oracle_attn(ctypes.byref(d), pre, cq, ckv, m, q.ctypes.data,
+                                  k.ctypes.data, v.ctypes.data, o.ctypes.data, lse.ctypes.data)
+    else:
+        sl = np.ascontiguousarray(np.asarray(slopes, dtype=np.float64).reshape(-1))
+        assert sl.shape == (pb.N,)
+        err = _load().oracle_attn_alibi(ctypes.byref(d), pre, cq, ckv, m, ALIBI[alibi],
+                                        sl.ctypes.data, q.ctypes.data, k.ctypes.data,
+                                        v.ctypes.data, o.ctypes.data, lse.ctypes.data)
     if err:
         raise MemoryError("oracle_attn: allocation failed")
     return o, lse

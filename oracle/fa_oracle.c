@@ -24,6 +24,11 @@
  *   - The same forward with keys and values read from paged caches (the
  *     "Norm" layout of the aclnnScatterPaKvCache page, scenario 2) through
  *     a per-sequence block table.
+ *   - An optional ALiBi bias added to the scores of the visible pairs, as
+ *     the Ascend ATB page "压缩mask" (alibi section) decomposes the alibi
+ *     mask: a per-head coefficient (slopes) times an alibi bias, plus the
+ *     triangular mask. Three biases, one per variant of that section:
+ *     right-aligned, its square root, and left-aligned.
  *   - The tiled online-softmax recurrence (running max m_i, running sum l_i,
  *     normalised output) of the "FlashAttention tiling & online softmax"
  *     exercise page (section "Mục tiêu kiến thức"), used only to pin the
@@ -41,6 +46,14 @@
  *   - Cumulative length arrays hold end offsets without a leading 0.
  *   - mode 0 without a mask computes everything (pre/next ignored); with a
  *     mask, the band AND the mask decide.
+ *   - ALiBi (the page's formula and figures are lost): the right-aligned
+ *     bias is the key's signed distance from the row's bottom-right-anchored
+ *     diagonal, j - (i + Skv_b - Sq_b), 0 on the diagonal and negative to
+ *     its left; the square-root variant takes the square root of that
+ *     distance's size and keeps its sign; the left-aligned bias is the key
+ *     position j itself (it differs from the right-aligned one by a
+ *     constant per row, so only lse moves). The score is
+ *     scale * q.k + slope_h * bias.
  *
  * Parity status: every function here is pinned by the CPU tests
  * (tests/test_oracle_pins.py) against library routines, closed forms and the
@@ -210,16 +223,39 @@ static int64_t lse_offset(const oracle_desc* d, int64_t b, int64_t h,
     return (b * d->N + h) * d->Sq + t;             /* [B, N, Sq] */
 }
 
+/* ALiBi variants (the three biases of the "压缩mask" page's alibi
+ * section). */
+enum { OR_ALIBI_NONE = 0, OR_ALIBI_RIGHT = 1, OR_ALIBI_SQRT = 2, OR_ALIBI_LEFT = 3 };
+
+/* The alibi bias of query i and key j of a sequence with sq rows and skv
+ * keys (positions inside the sequence). */
+static double alibi_bias(int kind, int64_t i, int64_t j, int64_t sq, int64_t skv) {
+    /* signed distance from the diagonal anchored at the bottom-right corner */
+    const double dist = (double)(j - (i + (skv - sq)));
+    switch (kind) {
+    case OR_ALIBI_RIGHT:
+        return dist;
+    case OR_ALIBI_SQRT:
+        return dist < 0 ? -sqrt(-dist) : sqrt(dist);
+    case OR_ALIBI_LEFT:
+        return (double)j;
+    default:
+        return 0.0;
+    }
+}
+
 /*
  * One query row of the plain attention definition:
- *   s_j = scale * sum_d q_d k_jd for the visible j, m = max s_j,
- *   l = sum exp(s_j - m), o = sum exp(s_j - m) v_j / l, lse = m + ln l.
- * vis_row holds the explicit visibility of the row's keys.
+ *   s_j = scale * sum_d q_d k_jd (+ bias_row[j]) for the visible j,
+ *   m = max s_j, l = sum exp(s_j - m), o = sum exp(s_j - m) v_j / l,
+ *   lse = m + ln l.
+ * vis_row holds the explicit visibility of the row's keys; bias_row (or
+ * NULL) an additive term per key.
  */
 static void attend_row(const oracle_desc* d, const double* q, const double* k,
                        const double* v, int64_t b, int64_t h, seq_info s,
-                       int64_t i, const uint8_t* vis_row, double* scores,
-                       double* o_row, double* lse_out) {
+                       int64_t i, const uint8_t* vis_row, const double* bias_row,
+                       double* scores, double* o_row, double* lse_out) {
     const int64_t D = d->D;
     const double* qi = q + row_offset(d, d->Sq, b, h, s.q_off + i);
     double m = -INFINITY;
@@ -228,7 +264,7 @@ static void attend_row(const oracle_desc* d, const double* q, const double* k,
         const double* kj = k + row_offset(d, d->Skv, b, h, s.kv_off + j);
         double acc = 0.0;
         for (int64_t x = 0; x < D; ++x) acc += qi[x] * kj[x];
-        scores[j] = d->scale * acc;
+        scores[j] = d->scale * acc + (bias_row ? bias_row[j] : 0.0);
         if (scores[j] > m) m = scores[j];
     }
     for (int64_t x = 0; x < D; ++x) o_row[x] = 0.0;
@@ -249,14 +285,17 @@ static void attend_row(const oracle_desc* d, const double* q, const double* k,
 }
 
 /*
- * Full forward: O (same layout as Q) and lse for every (b, h, row).
- * For each (b, h) the explicit Sq_b x Skv_b boolean visibility matrix is
- * built first, then the plain softmax is applied row by row.
+ * Full forward with an optional ALiBi bias: O (same layout as Q) and lse for
+ * every (b, h, row). For each (b, h) the explicit Sq_b x Skv_b boolean
+ * visibility matrix is built first, then the plain softmax is applied row by
+ * row, each visible score plus slopes[h] * alibi_bias(...) when alibi_kind
+ * is not OR_ALIBI_NONE (slopes: [N]).
  */
-int oracle_attn(const oracle_desc* d, const int64_t* prefix,
-                const int64_t* cu_q, const int64_t* cu_kv,
-                const uint8_t* mask, const double* q, const double* k,
-                const double* v, double* o, double* lse) {
+int oracle_attn_alibi(const oracle_desc* d, const int64_t* prefix,
+                      const int64_t* cu_q, const int64_t* cu_kv,
+                      const uint8_t* mask, int32_t alibi_kind,
+                      const double* slopes, const double* q, const double* k,
+                      const double* v, double* o, double* lse) {
     const int64_t nb = d->B, nh = d->N;
     int err = 0;
 #pragma omp parallel for collapse(2) schedule(dynamic, 1)
@@ -267,9 +306,11 @@ int oracle_attn(const oracle_desc* d, const int64_t* prefix,
             int64_t skv_alloc = s.skv > 0 ? s.skv : 1;
             uint8_t* vis = (uint8_t*)malloc((size_t)(s.sq * skv_alloc));
             double* scores = (double*)malloc(sizeof(double) * skv_alloc);
-            if (!vis || !scores) {
+            double* bias = (double*)malloc(sizeof(double) * skv_alloc);
+            if (!vis || !scores || !bias) {
                 free(vis);
                 free(scores);
+                free(bias);
 #pragma omp atomic write
                 err = 1;
                 continue;
@@ -280,14 +321,28 @@ int oracle_attn(const oracle_desc* d, const int64_t* prefix,
                         d, prefix, cu_q, cu_kv, mask, b, h, i, j);
             for (int64_t i = 0; i < s.sq; ++i) {
                 double* o_row = o + row_offset(d, d->Sq, b, h, s.q_off + i);
+                if (alibi_kind != OR_ALIBI_NONE)
+                    for (int64_t j = 0; j < s.skv; ++j)
+                        bias[j] = slopes[h] * alibi_bias(alibi_kind, i, j, s.sq, s.skv);
                 attend_row(d, q, k, v, b, h, s, i, vis + i * skv_alloc,
-                           scores, o_row, lse + lse_offset(d, b, h, s.q_off + i));
+                           alibi_kind != OR_ALIBI_NONE ? bias : NULL, scores,
+                           o_row, lse + lse_offset(d, b, h, s.q_off + i));
             }
             free(vis);
             free(scores);
+            free(bias);
         }
     }
     return err;
+}
+
+/* The forward without a bias. */
+int oracle_attn(const oracle_desc* d, const int64_t* prefix,
+                const int64_t* cu_q, const int64_t* cu_kv,
+                const uint8_t* mask, const double* q, const double* k,
+                const double* v, double* o, double* lse) {
+    return oracle_attn_alibi(d, prefix, cu_q, cu_kv, mask, OR_ALIBI_NONE, NULL,
+                             q, k, v, o, lse);
 }
 
 /*
@@ -317,7 +372,7 @@ int oracle_attn_rows(const oracle_desc* d, const int64_t* prefix,
         for (int64_t j = 0; j < s.skv; ++j)
             vis[j] = (uint8_t)oracle_visible(d, prefix, cu_q, cu_kv, mask, b,
                                              h, i, j);
-        attend_row(d, q, k, v, b, h, s, i, vis, scores, o_rows + r * d->D,
+        attend_row(d, q, k, v, b, h, s, i, vis, NULL, scores, o_rows + r * d->D,
                    lse_rows + r);
         free(vis);
         free(scores);

@@ -688,3 +688,124 @@ def test_tile_ranges_properties_on_random_class_rows(seed):
         longest = max(e - s for s, e in runs)
         assert fhi - flo == longest
         assert all(s >= flo for s, e in runs if e - s == longest)
+
+
+# --------------------------------------------------------------------------
+# ALiBi bias ("压缩mask" page, alibi section): per-head coefficient (slope)
+# times a bias, plus the triangular mask. Readings: right-aligned bias =
+# signed distance of key j from the row's bottom-right-anchored diagonal;
+# sqrt variant = the square root of that distance's size, sign kept;
+# left-aligned bias = j.
+# --------------------------------------------------------------------------
+
+ALIBI_SLOPES = [0.5, 0.125]
+
+
+def _zero_qk_identity_v(Sq, Skv, N):
+    """Q = K = 0 (every visible score is the bias alone) and V[j] = e_j, so
+    O[i, j] is the softmax weight of key j in row i."""
+    D = Skv
+    q = np.zeros((1, N, Sq, D))
+    k = np.zeros((1, N, Skv, D))
+    v = np.zeros((1, N, Skv, D))
+    for h in range(N):
+        v[0, h, np.arange(Skv), np.arange(Skv)] = 1.0
+    return q, k, v
+
+
+@pytest.mark.parametrize("Sq,Skv", [(5, 9), (7, 7)])
+def test_alibi_right_aligned_is_a_geometric_series(Sq, Skv):
+    """rightDownCausal with zero scores: row i sees n = i + delta + 1 keys with
+    weights exp(-a m), m = i + delta - j = 0..n-1, so lse = ln((1 - e^{-an}) /
+    (1 - e^{-a})) and O[i, j] = e^{-a m} (1 - e^{-a}) / (1 - e^{-an})."""
+    N = len(ALIBI_SLOPES)
+    q, k, v = _zero_qk_identity_v(Sq, Skv, N)
+    pb = Problem("BNSD", 1, N, Sq, Skv, Skv, sparse_mode=3)
+    o, lse = oracle.attention(pb, q, k, v, alibi="right", slopes=ALIBI_SLOPES)
+    delta = Skv - Sq
+    for h, a in enumerate(ALIBI_SLOPES):
+        for i in range(Sq):
+            n = i + delta + 1
+            assert lse[0, h, i] == pytest.approx(np.log((1 - np.exp(-a * n)) / (1 - np.exp(-a))),
+                                                 abs=1e-13)
+            want = np.zeros(Skv)
+            m = i + delta - np.arange(n)
+            want[:n] = np.exp(-a * m) * (1 - np.exp(-a)) / (1 - np.exp(-a * n))
+            np.testing.assert_allclose(o[0, h, i], want, rtol=0, atol=1e-14)
+
+
+def test_alibi_sqrt_equals_right_aligned_at_unit_distances():
+    """A band one key wide on each side of the diagonal (pre = 1, next = 1)
+    holds distances -1, 0, 1 only, whose square roots are themselves: the two
+    variants agree there; at larger distances they do not."""
+    Sq, Skv, D, N = 9, 12, 8, 2
+    q, k, v = _rand((1, N, Sq, D), 61), _rand((1, N, Skv, D), 62), _rand((1, N, Skv, D), 63)
+    pb = Problem("BNSD", 1, N, Sq, Skv, D, sparse_mode=4, pre_tokens=1, next_tokens=1)
+    o_r, l_r = oracle.attention(pb, q, k, v, alibi="right", slopes=ALIBI_SLOPES)
+    o_s, l_s = oracle.attention(pb, q, k, v, alibi="sqrt", slopes=ALIBI_SLOPES)
+    np.testing.assert_allclose(o_s, o_r, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(l_s, l_r, rtol=0, atol=1e-14)
+    wide = Problem("BNSD", 1, N, Sq, Skv, D, sparse_mode=3)
+    assert not np.allclose(oracle.attention(wide, q, k, v, alibi="sqrt", slopes=ALIBI_SLOPES)[1],
+                           oracle.attention(wide, q, k, v, alibi="right", slopes=ALIBI_SLOPES)[1])
+
+
+def test_alibi_sqrt_on_zero_scores():
+    """rightDownCausal with zero scores and the square-root bias: weights
+    exp(-a sqrt(m)) over m = 0..n-1."""
+    Sq, Skv = 6, 8
+    N = len(ALIBI_SLOPES)
+    q, k, v = _zero_qk_identity_v(Sq, Skv, N)
+    pb = Problem("BNSD", 1, N, Sq, Skv, Skv, sparse_mode=3)
+    o, lse = oracle.attention(pb, q, k, v, alibi="sqrt", slopes=ALIBI_SLOPES)
+    for h, a in enumerate(ALIBI_SLOPES):
+        for i in range(Sq):
+            n = i + (Skv - Sq) + 1
+            w = np.exp(-a * np.sqrt(np.arange(n)[::-1].astype(float)))
+            assert lse[0, h, i] == pytest.approx(np.log(w.sum()), abs=1e-13)
+            np.testing.assert_allclose(o[0, h, i, :n], w / w.sum(), rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("mode,extra", [(3, {}), (2, {}), (4, dict(pre_tokens=4, next_tokens=2)),
+                                        (0, {})])
+def test_alibi_left_aligned_moves_only_lse(mode, extra):
+    """Left- and right-aligned biases differ by slope * (i + delta) in each
+    row, a constant the softmax removes: O is the same, lse moves by it."""
+    Sq, Skv, D, N = 7, 10, 8, 2
+    q, k, v = _rand((1, N, Sq, D), 71), _rand((1, N, Skv, D), 72), _rand((1, N, Skv, D), 73)
+    pb = Problem("BNSD", 1, N, Sq, Skv, D, sparse_mode=mode, **extra)
+    o_r, l_r = oracle.attention(pb, q, k, v, alibi="right", slopes=ALIBI_SLOPES)
+    o_l, l_l = oracle.attention(pb, q, k, v, alibi="left", slopes=ALIBI_SLOPES)
+    np.testing.assert_allclose(o_l, o_r, rtol=0, atol=1e-13)
+    for h, a in enumerate(ALIBI_SLOPES):
+        np.testing.assert_allclose(l_l[0, h] - l_r[0, h], a * (np.arange(Sq) + Skv - Sq),
+                                   rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode,extra", [(3, {}), (0, {}), (5, dict(prefix=[4]))])
+def test_alibi_matches_sdpa_with_an_additive_mask(mode, extra):
+    """torch SDPA (fp64) with a float attn_mask: slope * bias on visible pairs
+    and -inf elsewhere, added to the scaled scores (the bias is not scaled);
+    keys right of the diagonal (mode 0, the prefix) get a positive bias."""
+    Sq, Skv, D, N = 6, 11, 8, 2
+    q, k, v = _rand((1, N, Sq, D), 81), _rand((1, N, Skv, D), 82), _rand((1, N, Skv, D), 83)
+    pb = Problem("BNSD", 1, N, Sq, Skv, D, sparse_mode=mode, **extra)
+    vis = oracle.mask_matrix(pb, 0).astype(bool)
+    dist = np.arange(Skv)[None, :] - (np.arange(Sq)[:, None] + Skv - Sq)
+    add = np.stack([np.where(vis, a * dist, -np.inf) for a in ALIBI_SLOPES])[None]
+    want = torch.nn.functional.scaled_dot_product_attention(
+        q, k, v, attn_mask=torch.from_numpy(add), scale=pb.scale).numpy()
+    o, lse = oracle.attention(pb, q, k, v, alibi="right", slopes=ALIBI_SLOPES)
+    np.testing.assert_allclose(o, want, rtol=0, atol=1e-12)
+    s = np.einsum("bhid,bhjd->bhij", q.numpy(), k.numpy()) * pb.scale + add
+    np.testing.assert_allclose(lse, torch.logsumexp(torch.from_numpy(s), -1).numpy(), atol=1e-12)
+
+
+def test_alibi_with_zero_slopes_is_the_plain_forward():
+    Sq, Skv, D, N = 9, 9, 8, 2
+    q, k, v = _rand((1, N, Sq, D), 91), _rand((1, N, Skv, D), 92), _rand((1, N, Skv, D), 93)
+    pb = Problem("BNSD", 1, N, Sq, Skv, D, sparse_mode=2)
+    o0, l0 = oracle.attention(pb, q, k, v)
+    for kind in ("right", "sqrt", "left"):
+        o, lse = oracle.attention(pb, q, k, v, alibi=kind, slopes=[0.0, 0.0])
+        assert np.array_equal(o, o0) and np.array_equal(lse, l0)
