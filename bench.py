@@ -163,11 +163,12 @@ def kernel_label(w, dense, dev):
     import torch
     import masked_attention_fa_b200 as fa
     d = fa.make_desc(w.layout, w.B, w.N, w.Sq, w.Skv, w.D, w.sparse_mode, w.pre_tokens,
-                     w.next_tokens, w.scale, w.mask_kind)
+                     w.next_tokens, w.scale, w.mask_kind, w.alibi)
     items = fa.fa_plan_stats(d, has_mask=dense, **workload_args(w))[0]
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     claim = (not dense) and items >= fa.CLAIM_MIN_ITEMS_PER_CTA * sms
-    return f"fa_fwd_sm100<{w.D}, true, {'true' if dense else 'false'}, {'true' if claim else 'false'}>"
+    tf = lambda x: "true" if x else "false"
+    return (f"fa_fwd_sm100<{w.D}, true, {tf(dense)}, {tf(claim)}, {tf(w.alibi is not None)}>")
 
 
 def visible_pairs(w, has_mask, mask_host=None):
@@ -260,6 +261,7 @@ def cpu_baseline_sample(w, inputs, seconds):
     import numpy as np
     import oracle
     from oracle import Problem
+    from masked_attention_fa_b200.workloads import alibi_slopes
     pb_kw = dict(layout=w.layout, B=w.B, N=w.N, Sq=w.Sq, Skv=w.Skv, D=w.D,
                  sparse_mode=w.sparse_mode, pre_tokens=w.pre_tokens, next_tokens=w.next_tokens,
                  scale=w.scale)
@@ -292,7 +294,11 @@ def cpu_baseline_sample(w, inputs, seconds):
         rows_i = rng.integers(0, nrows_total, size=chunk)
         rows = np.stack([np.zeros(chunk, np.int64), np.zeros(chunk, np.int64), rows_i], 1)
         t0 = time.perf_counter()
-        oracle.attention_rows(pb, qd, kd, vd, rows)
+        if w.alibi is not None:
+            oracle.attention_rows(pb, qd, kd, vd, rows, alibi=w.alibi,
+                                  slopes=alibi_slopes(w.N)[h:h + 1])
+        else:
+            oracle.attention_rows(pb, qd, kd, vd, rows)
         elapsed += time.perf_counter() - t0
         pairs += int(row_pairs[rows_i].sum())
         done_rows += chunk
@@ -311,6 +317,7 @@ def bench_config(w, pairs, world):
             "per_rank": "independent copy",
             "l2": "cold: a 256 MiB buffer is written between timed GPU steps",
             **({"block_size": w.block_size, "kv_cache": "paged, resident"} if paged else {}),
+            **({"alibi": w.alibi, "slopes": "2^(-8 (h + 1) / N), resident"} if w.alibi else {}),
             "parallelism": f"replicas x{world}"}
 
 
@@ -405,7 +412,11 @@ def main():
     mask = inputs["mask"].to(dev) if inputs["mask"] is not None else None
     arrays = workload_args(w)
     attn = fa.MaskedAttention(w.layout, w.B, w.N, w.Sq, w.Skv, w.D, w.sparse_mode, w.pre_tokens,
-                              w.next_tokens, w.scale, w.mask_kind)
+                              w.next_tokens, w.scale, w.mask_kind, w.alibi)
+    slopes = None
+    if w.alibi is not None:  # per-head coefficients: parameters, resident on the device
+        from masked_attention_fa_b200.workloads import alibi_slopes
+        slopes = torch.tensor(alibi_slopes(w.N), dtype=torch.float32, device=dev)
     oshape, lshape = attn.out_shapes()
     o = torch.empty(oshape, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(lshape, dtype=torch.float32, device=dev)
@@ -433,7 +444,8 @@ def main():
         elif dense:
             attn(q, k, v, atten_mask=mask, out=o, lse=lse, stream=stream, ranges=ranges)
         else:
-            attn(q, k, v, atten_mask=mask, out=o, lse=lse, stream=stream, **arrays)
+            attn(q, k, v, atten_mask=mask, out=o, lse=lse, stream=stream, slopes=slopes,
+                 **arrays)
 
     def step():
         if dense:
@@ -523,7 +535,7 @@ def main():
                 qb, kb, vb = dev_in[b][:3]
                 mb = dev_in[b][3] if dense else None
                 attn(qb, kb, vb, atten_mask=mb, out=dev_o[b], lse=dev_l[b], stream=stream,
-                     **arrays)
+                     slopes=slopes, **arrays)
             ev_fwd[b].record(stream)
             with torch.cuda.stream(down):
                 down.wait_event(ev_fwd[b])

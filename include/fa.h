@@ -70,13 +70,33 @@ typedef enum {
     FA_ERR_DEVICE = 8          /* the kernel reported an internal error */
 } fa_status_t;
 
+/* ALiBi bias added to the scores (the Ascend ATB page "压缩mask", alibi
+ * section: the alibi mask is a per-head coefficient, slopes[h], times an
+ * alibi bias, plus the triangular mask, in a right-aligned, a square-root and
+ * a left-aligned variant). The page's formula is lost; the reading taken, with
+ * delta_b = Skv_b - Sq_b and positions inside the sequence:
+ *   FA_ALIBI_RIGHT  bias(i, j) = j - (i + delta_b): the key's signed distance
+ *                   from the row's diagonal anchored at the bottom-right
+ *                   corner (0 on it, negative to its left);
+ *   FA_ALIBI_SQRT   the square root of that distance's size, sign kept;
+ *   FA_ALIBI_LEFT   bias(i, j) = j (a constant per row away from RIGHT: the
+ *                   same O, lse larger by slopes[h] * (i + delta_b)).
+ * The score of a visible pair is scale * q.k + slopes[h] * bias(i, j); the
+ * visibility rule is the sparseMode geometry, unchanged. */
+typedef enum {
+    FA_ALIBI_NONE = 0,
+    FA_ALIBI_RIGHT = 1,
+    FA_ALIBI_SQRT = 2,
+    FA_ALIBI_LEFT = 3
+} fa_alibi_t;
+
 /* Problem descriptor. For FA_TND, B is the number of sequences and Sq / Skv
  * are the token totals T_q / T_kv. */
 typedef struct {
     int32_t layout;        /* fa_layout_t */
     int32_t sparse_mode;   /* 0..8 */
     int32_t mask_kind;     /* fa_mask_kind_t; must be NONE unless mode 0/1 */
-    int32_t reserved;      /* must be 0 */
+    int32_t alibi;         /* fa_alibi_t; FA_ALIBI_NONE (0) unless the call is fa_fwd_alibi */
     int64_t B, N, Sq, Skv, D;
     int64_t pre_tokens;    /* preTokens  (modes 0, 4, 7, 8; ignored otherwise) */
     int64_t next_tokens;   /* nextTokens (modes 0, 4, 7, 8; ignored otherwise) */
@@ -95,7 +115,9 @@ typedef struct {
  *   gives no TND mask shape); modes 7 and 8 need TND; in mode 0 with a mask,
  *   next < 0 needs pre >= |next| and |next| < Skv, pre < 0 needs
  *   next >= |pre| and |pre| < Sq (sparseMode=0 section, the two 说明 notes);
- *   in mode 4 the band must intersect: pre + next >= 0 (sparseMode=4).
+ *   in mode 4 the band must intersect: pre + next >= 0 (sparseMode=4);
+ *   alibi in 0..3, and an ALiBi bias only without an attenMask (mask_kind
+ *   NONE; FA_ERR_UNSUPPORTED otherwise).
  * Ownership: the handle owns a small device workspace (work list, counters,
  * error word) and a pinned staging buffer, released by fa_destroy. The
  * workspace is allocated on the current device at the first fa_fwd.
@@ -154,6 +176,24 @@ fa_status_t fa_fwd(fa_handle_t h, const void* q, const void* k, const void* v,
                    const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
                    void* o, float* lse, void* cuda_stream);
 
+/*
+ * fa_fwd_alibi — fa_fwd for a handle whose descriptor names an ALiBi
+ * variant (alibi != FA_ALIBI_NONE): every visible score gets
+ * slopes[h] * bias(i, j) added before the softmax (see fa_alibi_t).
+ *
+ * slopes  device fp32 [N], 4-byte aligned, finite; read by the kernel.
+ * The other arguments and the asynchronous behaviour are fa_fwd's. Errors:
+ * FA_ERR_NULLPTR (NULL slopes), FA_ERR_PARAM_INVALID (a handle without an
+ * ALiBi variant, unaligned slopes), and fa_fwd's. fa_fwd on an ALiBi handle
+ * returns FA_ERR_PARAM_INVALID (it has no slopes). The lse is fp32: in the
+ * left-aligned variant it grows like slopes[h] * (i + delta_b), and its
+ * absolute rounding error with it.
+ */
+fa_status_t fa_fwd_alibi(fa_handle_t h, const void* q, const void* k, const void* v,
+                         const float* slopes, const int64_t* prefix,
+                         const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
+                         void* o, float* lse, void* cuda_stream);
+
 /* fa_sync_status — wait for the handle's last call and read its device error
  * word: FA_OK, FA_ERR_TIMEOUT (a bounded wait in the kernel gave up, its
  * outputs are undefined) or FA_ERR_DEVICE. The error word is cleared. */
@@ -178,7 +218,8 @@ int32_t fa_version(void);
  * memory callbacks). The pages have no counterpart of this entry point.
  *
  * No handle: the descriptor and all arrays are passed on every call, with
- * the meaning, layout and validation of fa_create + fa_fwd. The work list
+ * the meaning, layout and validation of fa_create + fa_fwd. A descriptor
+ * with an ALiBi variant is FA_ERR_UNSUPPORTED here (there are no slopes). The work list
  * and the error word live in one fixed device array of 1 MiB per device,
  * held from library load until process exit, instead of a cudaMalloc'd
  * workspace: the call makes no cudaMalloc, cudaFree or pinned allocation.
@@ -257,7 +298,7 @@ fa_status_t fa_noalloc_sync_status(void* cuda_stream);
  * Visibility: the handle's sparseMode row intervals per sequence (modes 0
  * without a mask, 2..8), exactly as fa_fwd applies them to TND.
  * Constraints (FA_ERR_* before any device work): a TND handle with no mask
- * kind and sparse_mode != 1; 1 <= block_size <= 2^20; num_blocks >= 1;
+ * kind, no ALiBi variant and sparse_mode != 1; 1 <= block_size <= 2^20; num_blocks >= 1;
  * ceil(Skv_b / block_size) <= max_blocks for every b.
  * The work is split over the keys (units of one sequence, one head, up to 4
  * query rows and one chunk of keys) and each row's chunks are merged in a

@@ -26,6 +26,9 @@ STATUS = {0: "FA_OK", 1: "FA_ERR_NULLPTR", 2: "FA_ERR_PARAM_INVALID", 3: "FA_ERR
           4: "FA_ERR_UNSUPPORTED", 5: "FA_ERR_ALLOC", 6: "FA_ERR_CUDA", 7: "FA_ERR_TIMEOUT",
           8: "FA_ERR_DEVICE"}
 FA_TILE_EMPTY, FA_TILE_PARTIAL, FA_TILE_FULL = 0, 1, 2
+FA_ALIBI_NONE, FA_ALIBI_RIGHT, FA_ALIBI_SQRT, FA_ALIBI_LEFT = 0, 1, 2, 3
+ALIBI = {None: FA_ALIBI_NONE, "right": FA_ALIBI_RIGHT, "sqrt": FA_ALIBI_SQRT,
+         "left": FA_ALIBI_LEFT}
 
 
 class FaError(RuntimeError):
@@ -40,7 +43,7 @@ class fa_desc_t(ctypes.Structure):
         ("layout", ctypes.c_int32),
         ("sparse_mode", ctypes.c_int32),
         ("mask_kind", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("alibi", ctypes.c_int32),
         ("B", ctypes.c_int64),
         ("N", ctypes.c_int64),
         ("Sq", ctypes.c_int64),
@@ -82,6 +85,8 @@ def load_library():
     lib.fa_create.restype = st
     lib.fa_fwd.argtypes = [P, P, P, P, P, i64p, i64p, i64p, P, P, P]
     lib.fa_fwd.restype = st
+    lib.fa_fwd_alibi.argtypes = [P, P, P, P, P, i64p, i64p, i64p, P, P, P]
+    lib.fa_fwd_alibi.restype = st
     lib.fa_sync_status.argtypes = [P]
     lib.fa_sync_status.restype = st
     lib.fa_destroy.argtypes = [P]
@@ -123,7 +128,7 @@ def load_library():
 EXPORTED = ("fa_create", "fa_fwd", "fa_sync_status", "fa_destroy", "fa_last_error",
             "fa_version", "fa_validate", "fa_visible_pairs", "fa_tile_class", "fa_plan_stats",
             "fa_plan_items", "fa_fwd_noalloc", "fa_split_queries", "fa_mask_occupancy",
-            "fa_fwd_with_ranges", "fa_fwd_paged", "fa_noalloc_sync_status")
+            "fa_fwd_with_ranges", "fa_fwd_paged", "fa_noalloc_sync_status", "fa_fwd_alibi")
 
 
 def _check(status):
@@ -139,11 +144,12 @@ CLAIM_MIN_ITEMS_PER_CTA = 8
 
 
 def make_desc(layout, B, N, Sq, Skv, D, sparse_mode=0, pre_tokens=0, next_tokens=0, scale=None,
-              mask_kind=None) -> fa_desc_t:
+              mask_kind=None, alibi=None) -> fa_desc_t:
     lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
     mk = MASK_KINDS[mask_kind] if (mask_kind is None or isinstance(mask_kind, str)) else int(mask_kind)
+    al = ALIBI[alibi] if (alibi is None or isinstance(alibi, str)) else int(alibi)
     sc = (1.0 / float(D) ** 0.5) if scale is None else float(scale)
-    return fa_desc_t(lay, int(sparse_mode), mk, 0, int(B), int(N), int(Sq), int(Skv), int(D),
+    return fa_desc_t(lay, int(sparse_mode), mk, al, int(B), int(N), int(Sq), int(Skv), int(D),
                      int(pre_tokens), int(next_tokens), sc)
 
 
@@ -254,6 +260,15 @@ def fa_fwd(h, q, k, v, o, lse, atten_mask=None, prefix=None, actual_seq_qlen=Non
     a = _Arrays(prefix, actual_seq_qlen, actual_seq_kvlen)
     _check(load_library().fa_fwd(h, _ptr(q), _ptr(k), _ptr(v), _ptr(atten_mask), *a.ptrs(),
                                  _ptr(o), _ptr(lse), ctypes.c_void_p(int(stream))))
+
+
+def fa_fwd_alibi(h, q, k, v, slopes, o, lse, prefix=None, actual_seq_qlen=None,
+                 actual_seq_kvlen=None, stream=None):
+    """fa_fwd for a handle with an ALiBi variant; slopes: fp32 CUDA tensor [N]."""
+    a = _Arrays(prefix, actual_seq_qlen, actual_seq_kvlen)
+    _check(load_library().fa_fwd_alibi(h, _ptr(q), _ptr(k), _ptr(v), _ptr(slopes), *a.ptrs(),
+                                       _ptr(o), _ptr(lse),
+                                       ctypes.c_void_p(_stream_int(stream, q.device))))
 
 
 def _stream_int(stream, device):
@@ -370,10 +385,10 @@ class MaskedAttention:
     """A handle for one problem shape: ``o, lse = attn(q, k, v, ...)``."""
 
     def __init__(self, layout, B, N, Sq, Skv, D, sparse_mode=0, pre_tokens=0, next_tokens=0,
-                 scale=None, mask_kind=None):
+                 scale=None, mask_kind=None, alibi=None):
         self.layout = layout
         self.desc = make_desc(layout, B, N, Sq, Skv, D, sparse_mode, pre_tokens, next_tokens,
-                              scale, mask_kind)
+                              scale, mask_kind, alibi)
         self.handle = fa_create(self.desc)
 
     def out_shapes(self):
@@ -385,7 +400,8 @@ class MaskedAttention:
         return (d.Sq, d.N, d.D), (d.N, d.Sq)
 
     def __call__(self, q, k, v, atten_mask=None, prefix=None, actual_seq_qlen=None,
-                 actual_seq_kvlen=None, out=None, lse=None, stream=None, ranges=None):
+                 actual_seq_kvlen=None, out=None, lse=None, stream=None, ranges=None,
+                 slopes=None):
         import torch
         oshape, lshape = self.out_shapes()
         if out is None:
@@ -400,7 +416,12 @@ class MaskedAttention:
         if atten_mask is not None:
             if atten_mask.dtype not in (torch.uint8, torch.bool) or not atten_mask.is_contiguous():
                 raise ValueError("atten_mask must be a contiguous uint8/bool tensor")
-        if ranges is not None:
+        if slopes is not None:
+            if slopes.dtype != torch.float32 or not slopes.is_contiguous() or not slopes.is_cuda:
+                raise ValueError("slopes must be a contiguous fp32 CUDA tensor")
+            fa_fwd_alibi(self.handle, q, k, v, slopes, out, lse, prefix, actual_seq_qlen,
+                         actual_seq_kvlen, stream)
+        elif ranges is not None:
             fa_fwd_with_ranges(self.handle, q, k, v, out, lse, atten_mask, ranges, stream)
         else:
             fa_fwd(self.handle, q, k, v, out, lse, atten_mask, prefix, actual_seq_qlen,

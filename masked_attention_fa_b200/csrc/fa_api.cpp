@@ -308,12 +308,17 @@ namespace {
 // fa_fwd and fa_fwd_with_ranges. `ranges` (or null): the dense-mask
 // occupancy of this mask, already computed by fa_mask_occupancy.
 fa_status_t forward(fa_handle_t h, const void* q, const void* k, const void* v,
-                    const uint8_t* atten_mask, const int32_t* ranges, const int64_t* prefix,
-                    const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen, void* o,
-                    float* lse, void* cuda_stream) {
+                    const uint8_t* atten_mask, const int32_t* ranges, const float* slopes,
+                    const int64_t* prefix, const int64_t* actual_seq_qlen,
+                    const int64_t* actual_seq_kvlen, void* o, float* lse, void* cuda_stream) {
   if (!h) return fail(FA_ERR_NULLPTR, "handle is NULL");
   if (!q || !k || !v || !o || !lse) return fail(FA_ERR_NULLPTR, "q, k, v, o and lse are required");
   const fa_desc_t* d = &h->desc;
+  if (d->alibi != FA_ALIBI_NONE && !slopes)
+    return fail(FA_ERR_PARAM_INVALID,
+                "the handle names an ALiBi variant: call fa_fwd_alibi with the slopes");
+  if (slopes && ((uintptr_t)slopes & 3u))
+    return fail(FA_ERR_PARAM_INVALID, "slopes must be 4-byte aligned");
   const int m = d->sparse_mode;
   const int has_mask = (m <= 1) && atten_mask != nullptr;
   fa_status_t st = validate_call(d, prefix, actual_seq_qlen, actual_seq_kvlen, has_mask);
@@ -408,6 +413,10 @@ fa_status_t forward(fa_handle_t h, const void* q, const void* k, const void* v,
     p.claim = reinterpret_cast<unsigned int*>(ws + kClaimOffset);
     p.claim_done = reinterpret_cast<unsigned int*>(ws + kClaimOffset + 64);
   }
+  if (d->alibi != FA_ALIBI_NONE) {
+    p.slopes = slopes;
+    p.alibi = d->alibi;
+  }
   p.tnd = d->layout == FA_TND ? 1 : 0;
   p.scale_log2 = (float)(d->scale * 1.4426950408889634073599);
   p.debug_flags = h->debug_flags;
@@ -434,8 +443,21 @@ fa_status_t fa_fwd(fa_handle_t h, const void* q, const void* k, const void* v,
                    const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen, void* o,
                    float* lse, void* cuda_stream) {
   clear_error();
-  return forward(h, q, k, v, atten_mask, nullptr, prefix, actual_seq_qlen, actual_seq_kvlen, o,
-                 lse, cuda_stream);
+  return forward(h, q, k, v, atten_mask, nullptr, nullptr, prefix, actual_seq_qlen,
+                 actual_seq_kvlen, o, lse, cuda_stream);
+}
+
+fa_status_t fa_fwd_alibi(fa_handle_t h, const void* q, const void* k, const void* v,
+                         const float* slopes, const int64_t* prefix,
+                         const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
+                         void* o, float* lse, void* cuda_stream) {
+  clear_error();
+  if (!h) return fail(FA_ERR_NULLPTR, "handle is NULL");
+  if (!slopes) return fail(FA_ERR_NULLPTR, "slopes is NULL");
+  if (h->desc.alibi == FA_ALIBI_NONE)
+    return fail(FA_ERR_PARAM_INVALID, "fa_fwd_alibi needs a handle with an ALiBi variant");
+  return forward(h, q, k, v, nullptr, nullptr, slopes, prefix, actual_seq_qlen,
+                 actual_seq_kvlen, o, lse, cuda_stream);
 }
 
 fa_status_t fa_fwd_with_ranges(fa_handle_t h, const void* q, const void* k, const void* v,
@@ -448,7 +470,8 @@ fa_status_t fa_fwd_with_ranges(fa_handle_t h, const void* q, const void* k, cons
                 "fa_fwd_with_ranges needs sparse_mode 0 or 1 with a mask kind and atten_mask");
   if (!ranges) return fail(FA_ERR_NULLPTR, "ranges is NULL");
   if ((uintptr_t)ranges & 15u) return fail(FA_ERR_PARAM_INVALID, "ranges must be 16-byte aligned");
-  return forward(h, q, k, v, atten_mask, ranges, nullptr, nullptr, nullptr, o, lse, cuda_stream);
+  return forward(h, q, k, v, atten_mask, ranges, nullptr, nullptr, nullptr, nullptr, o, lse,
+                 cuda_stream);
 }
 
 fa_status_t fa_fwd_paged(fa_handle_t h, const void* q, const void* k_cache, const void* v_cache,

@@ -42,6 +42,10 @@ struct __align__(64) FwdParams {
   // by descending cost), and calls that do not overlap on the GPU.
   unsigned int* claim;
   unsigned int* claim_done;
+  // ALiBi (or null): per-head slopes [N], fp32; alibi is the fa_alibi_t
+  // variant. Only the closed-form instances with item_tr add the bias.
+  const float* slopes;
+  int32_t alibi;
   int32_t n_items;
   int32_t tnd;             // packed tokens: TMA batch coordinate 0, token = offset + row
   float scale_log2;        // scale * log2(e)

@@ -921,6 +921,34 @@ __device__ __forceinline__ void exp_pack_part(const float (&x)[128], uint64_t m2
   }
 }
 
+// ALiBi: scores of the row's 128 keys of this tile in log2 units with the
+// bias added, x <- x * scale_log2 + a2 * bias, a2 = slope * log2(e). d0 is
+// the signed distance of the tile's first key from the row's diagonal
+// anchored at the bottom-right corner (key c is d0 + c away). The linear
+// bias (right-aligned; the left-aligned one differs by a constant per row,
+// applied to lse at the end) is a ramp with one FMA per key; the square-root
+// variant takes sqrt of each distance's size on the MUFU unit and keeps its
+// sign. Hidden keys stay -inf.
+__device__ __forceinline__ void apply_alibi(float (&x)[128], float scale_log2, float a2, int d0,
+                                            bool sqrt_bias) {
+  if (sqrt_bias) {
+#pragma unroll
+    for (int c = 0; c < 128; ++c) {
+      const float d = (float)(d0 + c);
+      float r;
+      asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(fabsf(d)));
+      x[c] = fmaf(x[c], scale_log2, a2 * copysignf(r, d));
+    }
+  } else {
+    const float base = a2 * (float)d0;
+    const uint64_t s2 = pack_f32x2(scale_log2, scale_log2);
+#pragma unroll
+    for (int c = 0; c < 128; c += 2)
+      fma_x2(x[c], x[c + 1], s2,
+             pack_f32x2(fmaf((float)c, a2, base), fmaf((float)(c + 1), a2, base)));
+  }
+}
+
 __device__ __forceinline__ float sum_acc(float (&acc)[8]) {
   add_x2(acc[0], acc[1], acc[2], acc[3]);
   add_x2(acc[4], acc[5], acc[6], acc[7]);
@@ -980,7 +1008,8 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // warpgroup.
 // kDense: the dense-mask extras (the next mask line prefetched a tile ahead,
 // 16-byte mask gathers), compiled only into the dense-mask instance.
-template <int D, bool kOcc, bool kDense, bool kClaim>
+// kAlibi: the ALiBi bias added to the scores before the row maximum.
+template <int D, bool kOcc, bool kDense, bool kClaim, bool kAlibi>
 __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, float* inv_l_sm,
                              uint32_t tmem, uint8_t* sP, int sub, const WaitCtx& w) {
   using C = Cfg<D>;
@@ -1028,6 +1057,15 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
     if (row_valid) {
       jlo = (int)imax64(0, row_lo(sr, i));
       jhi = (int)imin64((int64_t)sr.skv - 1, row_hi(sr, i));
+    }
+    // ALiBi: slope of the head, in log2 units, and the distance of key 0
+    // from this row's bottom-right-anchored diagonal.
+    float slope = 0.f, a2 = 0.f;
+    int dbase = 0;
+    if constexpr (kAlibi) {
+      slope = __ldg(p.slopes + it.h);
+      a2 = slope * 1.4426950408889634f;
+      dbase = -(i + (sr.skv - sr.sq));
     }
     const uint8_t* mrow = nullptr;
     if ((sr.flags & kSeqDenseMask) && row_valid)
@@ -1111,7 +1149,11 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
       // S_s is in registers: the next QK of this sub-tile may overwrite it.
       tc_fence_before();
       mbar_arrive(&ctl->s_free[sub]);
-      const float m_new = row_max128(x) * scale_log2;
+      // Without ALiBi the scale is applied inside the exponential (the max
+      // of the raw scores scales, scale > 0); with it x holds the biased
+      // scores in log2 units already.
+      if constexpr (kAlibi) apply_alibi(x, scale_log2, a2, t * kTileN + dbase, p.alibi == 2);
+      const float m_new = kAlibi ? row_max128(x) : row_max128(x) * scale_log2;
       const bool resc = m_new > m_used + kRescaleLog2;
       float alpha = 1.f;
       if (resc) {
@@ -1125,7 +1167,8 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
         break;
       }
       const float ref = ((m_used == -INFINITY) ? 0.f : m_used) + zero;
-      const uint64_t m2 = pack_f32x2(scale_log2, scale_log2);
+      const float mul = kAlibi ? 1.f : scale_log2;
+      const uint64_t m2 = pack_f32x2(mul, mul);
       const uint64_t c2 = pack_f32x2(-ref, -ref);
       uint32_t pk[64];
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -1193,7 +1236,11 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
     inv_l_sm[sub * kTileM + row] = l > 0.f ? rcp_fast(l) : 0.f;
     mbar_arrive(&ctl->epi_full[sub]);
     if (row_valid) {
-      const float lse = l > 0.f ? (m_used + lg2_fast(l)) * 0.69314718055994530942f : -INFINITY;
+      float lse = l > 0.f ? (m_used + lg2_fast(l)) * 0.69314718055994530942f : -INFINITY;
+      // Left-aligned ALiBi: the same weights, every score larger by
+      // slope * (i + Skv - Sq) than the right-aligned one computed here.
+      if constexpr (kAlibi)
+        if (p.alibi == 3 && l > 0.f) lse = fmaf(slope, (float)(-dbase), lse);
       st_global_na_f32(p.lse + it.b * p.l_sb + it.h * p.l_sh + sr.q_off + i, lse);
     }
   }
@@ -1263,7 +1310,7 @@ __device__ void epilogue_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl,
   }
 }
 
-template <int D, bool kOcc, bool kDense, bool kClaim>
+template <int D, bool kOcc, bool kDense, bool kClaim, bool kAlibi>
 __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100(const __grid_constant__ FwdParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -1324,7 +1371,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100(const __grid_constan
 
   if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-    softmax_role<D, kOcc, kDense, kClaim>(p, ctl, inv_l_sm, tmem, sP, warp >> 2, w);
+    softmax_role<D, kOcc, kDense, kClaim, kAlibi>(p, ctl, inv_l_sm, tmem, sP, warp >> 2, w);
   } else if (warp < 12) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
     epilogue_role<D, kOcc, kClaim>(p, ctl, inv_l_sm, tmem, w);
@@ -1393,10 +1440,10 @@ bool encode_operand_map(CUtensorMap* tm, const void* base, int64_t D, int64_t S,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool kOcc, bool kDense, bool kClaim = false>
+template <int D, bool kOcc, bool kDense, bool kClaim = false, bool kAlibi = false>
 static cudaError_t launch_d(const FwdParams& p, int grid, cudaStream_t stream, const char** why) {
   using C = dev::Cfg<D>;
-  auto kern = dev::fa_fwd_sm100<D, kOcc, kDense, kClaim>;
+  auto kern = dev::fa_fwd_sm100<D, kOcc, kDense, kClaim, kAlibi>;
   static bool configured = false;
   static bool regs_ok = false;
   if (!configured) {
@@ -1421,23 +1468,36 @@ static cudaError_t launch_d(const FwdParams& p, int grid, cudaStream_t stream, c
 
 cudaError_t launch_fwd(int D, const FwdParams& p, int grid, cudaStream_t stream,
                        const char** why) {
-  // Four instances per head dim: ranges beside the items with the
-  // dense-mask extras, without them (fixed snake or claimed work), and
-  // ranges from the closed form (no item_tr). Only the claiming instance
-  // reads p.claim.
+  // Six instances per head dim: ranges beside the items with the
+  // dense-mask extras, without them (fixed snake or claimed work, each also
+  // with the ALiBi bias), and ranges from the closed form (no item_tr). Only
+  // the claiming instances read p.claim.
   const bool occ = p.item_tr != nullptr;
   const bool dense = occ && p.mask != nullptr && p.m_si > 0;
   const bool claim = occ && !dense && p.claim != nullptr;
-  if (D == 128)
+  const bool alibi = p.slopes != nullptr;
+  if (alibi && (!occ || dense)) {
+    if (why) *why = "an ALiBi bias needs a closed-form call with per-item ranges";
+    return cudaErrorInvalidValue;
+  }
+  if (D == 128) {
+    if (alibi)
+      return claim ? launch_d<128, true, false, true, true>(p, grid, stream, why)
+                   : launch_d<128, true, false, false, true>(p, grid, stream, why);
     return dense   ? launch_d<128, true, true>(p, grid, stream, why)
            : claim ? launch_d<128, true, false, true>(p, grid, stream, why)
            : occ   ? launch_d<128, true, false>(p, grid, stream, why)
                    : launch_d<128, false, false>(p, grid, stream, why);
-  if (D == 64)
+  }
+  if (D == 64) {
+    if (alibi)
+      return claim ? launch_d<64, true, false, true, true>(p, grid, stream, why)
+                   : launch_d<64, true, false, false, true>(p, grid, stream, why);
     return dense   ? launch_d<64, true, true>(p, grid, stream, why)
            : claim ? launch_d<64, true, false, true>(p, grid, stream, why)
            : occ   ? launch_d<64, true, false>(p, grid, stream, why)
                    : launch_d<64, false, false>(p, grid, stream, why);
+  }
   if (why) *why = "unsupported head dim";
   return cudaErrorInvalidValue;
 }

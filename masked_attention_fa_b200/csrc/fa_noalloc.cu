@@ -158,6 +158,8 @@ extern "C" fa_status_t fa_fwd_noalloc(const fa_desc_t* desc, const void* q, cons
   const int has_mask = (desc->sparse_mode <= 1) && atten_mask != nullptr;
   fa_status_t st = validate_call(desc, prefix, actual_seq_qlen, actual_seq_kvlen, has_mask);
   if (st != FA_OK) return st;
+  if (desc->alibi != FA_ALIBI_NONE)
+    return fail(FA_ERR_UNSUPPORTED, "fa_fwd_noalloc takes no ALiBi slopes; use fa_fwd_alibi");
   const uintptr_t align = (uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)o;
   if (align & 15u) return fail(FA_ERR_PARAM_INVALID, "q, k, v and o must be 16-byte aligned");
   if ((uintptr_t)lse & 3u) return fail(FA_ERR_PARAM_INVALID, "lse must be 4-byte aligned");

@@ -44,7 +44,9 @@ fa_status_t validate_desc(const fa_desc_t* d) {
     return fail(FA_ERR_PARAM_INVALID, "layout %d is not BNSD(0), BSND(1) or TND(2)", d->layout);
   if (d->sparse_mode < 0 || d->sparse_mode > 8)
     return fail(FA_ERR_PARAM_INVALID, "sparse_mode %d is outside 0..8", d->sparse_mode);
-  if (d->reserved != 0) return fail(FA_ERR_PARAM_INVALID, "reserved field must be 0");
+  if (d->alibi < FA_ALIBI_NONE || d->alibi > FA_ALIBI_LEFT)
+    return fail(FA_ERR_PARAM_INVALID, "alibi %d is not NONE(0), RIGHT(1), SQRT(2) or LEFT(3)",
+                d->alibi);
   if (d->B < 1 || d->N < 1 || d->D < 1)
     return fail(FA_ERR_SHAPE, "B, N and D must be >= 1 (got %lld, %lld, %lld)", (long long)d->B,
                 (long long)d->N, (long long)d->D);
@@ -72,6 +74,8 @@ fa_status_t validate_desc(const fa_desc_t* d) {
                 "sparse_mode %d derives its mask from the geometry; mask_kind must be NONE", m);
   if (m == 1 && d->mask_kind == FA_MASK_NONE)
     return fail(FA_ERR_PARAM_INVALID, "sparse_mode 1 (allMask) needs a mask_kind");
+  if (d->alibi != FA_ALIBI_NONE && d->mask_kind != FA_MASK_NONE)
+    return fail(FA_ERR_UNSUPPORTED, "an ALiBi bias with an attenMask is not supported");
   if (d->layout == FA_TND && d->mask_kind != FA_MASK_NONE)
     return fail(FA_ERR_UNSUPPORTED, "an attenMask with the TND layout is not supported");
   if ((m == 7 || m == 8) && d->layout != FA_TND)
@@ -280,6 +284,8 @@ fa_status_t validate_paged(const fa_desc_t* d, const int64_t* prefix, const int6
     return fail(FA_ERR_UNSUPPORTED, "paged K/V needs a TND handle (packed query tokens)");
   if (d->sparse_mode == 1 || d->mask_kind != FA_MASK_NONE)
     return fail(FA_ERR_UNSUPPORTED, "paged K/V reads no attenMask (dense-mask modes need BNSD/BSND)");
+  if (d->alibi != FA_ALIBI_NONE)
+    return fail(FA_ERR_UNSUPPORTED, "paged K/V does not add an ALiBi bias");
   if (block_size < 1 || block_size > (1 << 20))
     return fail(FA_ERR_PARAM_INVALID, "block_size %d outside [1, 2^20]", block_size);
   if (max_blocks < 1) return fail(FA_ERR_PARAM_INVALID, "max_blocks %d < 1", max_blocks);

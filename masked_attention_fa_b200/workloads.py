@@ -46,6 +46,7 @@ class Workload:
     actual_seq_kvlen: Optional[list] = None
     scale: Optional[float] = None
     block_size: Optional[int] = None     # paged K/V caches of this block size (TND queries)
+    alibi: Optional[str] = None          # ALiBi variant ("right", "sqrt", "left") or None
 
     def __post_init__(self):
         if self.scale is None:
@@ -99,6 +100,13 @@ def varlen_lengths(gen: torch.Generator, nseq: int, q_lo: int, q_hi: int, extra_
     extra = torch.randint(0, extra_hi + 1, (nseq,), generator=gen)
     skv = sq + extra
     return torch.cumsum(sq, 0).tolist(), torch.cumsum(skv, 0).tolist()
+
+
+def alibi_slopes(N: int):
+    """Per-head ALiBi coefficients for N heads, the geometric sequence
+    2^(-8 (h + 1) / N), h = 0..N-1, as synthetic inputs (the compressed-mask
+    page passes slopes in but does not say how they are chosen)."""
+    return [2.0 ** (-8.0 * (h + 1) / N) for h in range(N)]
 
 
 def lower_triangular_mask(S: int) -> torch.Tensor:
@@ -210,6 +218,10 @@ def named_workloads() -> dict:
                                            actual_seq_kvlen=cu_kv),
         "prefix_8k": Workload("prefix_8k", "BNSD", 4, 16, 8192, 8192, 128, 5, seed=5,
                               prefix=[512, 1024, 2048, 4096]),
+        # leftUpCausal with the right-aligned ALiBi bias of the compressed-mask
+        # page (slopes: alibi_slopes(16)); same shape and q, k, v as above
+        "alibi_causal_4k": Workload("alibi_causal_4k", "BNSD", 2, 16, 4096, 4096, 128, 2, seed=2,
+                                    alibi="right"),
         # the leftUpCausal problem (same shape and seed, so the same q, k, v)
         # given as an explicit lower-triangular allMask (sparseMode 1)
         "allmask_causal_4k": Workload("allmask_causal_4k", "BNSD", 2, 16, 4096, 4096, 128, 1,

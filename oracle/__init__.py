@@ -75,6 +75,9 @@ def _load():
         lib.oracle_attn_alibi.restype = ctypes.c_int
         lib.oracle_attn_rows.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, P, P, P, i64, P, P, P]
         lib.oracle_attn_rows.restype = ctypes.c_int
+        lib.oracle_attn_rows_alibi.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, ctypes.c_int32,
+                                               P, P, P, P, i64, P, P, P]
+        lib.oracle_attn_rows_alibi.restype = ctypes.c_int
         lib.oracle_mask.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, i64, i64, P]
         lib.oracle_mask.restype = None
         lib.oracle_tile_classes.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, i64, i64, i64, P]
@@ -261,8 +264,9 @@ def attention_paged(pb: Problem, q, k_cache, v_cache, block_table, block_size: i
     return o, lse
 
 
-def attention_rows(pb: Problem, q, k, v, rows):
-    """Selected rows (b, h, i) only: returns (O rows [n, D], lse [n])."""
+def attention_rows(pb: Problem, q, k, v, rows, alibi=None, slopes=None):
+    """Selected rows (b, h, i) only: returns (O rows [n, D], lse [n]); the
+    ALiBi arguments are attention()'s."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
     n = rows.shape[0]
@@ -270,9 +274,14 @@ def attention_rows(pb: Problem, q, k, v, rows):
     lse = np.zeros((n,), dtype=np.float64)
     d = pb.desc()
     pre, cq, ckv, m = pb._ptrs()
-    err = _load().oracle_attn_rows(ctypes.byref(d), pre, cq, ckv, m, q.ctypes.data, k.ctypes.data,
-                                   v.ctypes.data, n, rows.ctypes.data, o.ctypes.data,
-                                   lse.ctypes.data)
+    sl = None
+    if alibi is not None:
+        sl = np.ascontiguousarray(np.asarray(slopes, dtype=np.float64).reshape(-1))
+        assert sl.shape == (pb.N,)
+    err = _load().oracle_attn_rows_alibi(ctypes.byref(d), pre, cq, ckv, m, ALIBI[alibi],
+                                         None if sl is None else sl.ctypes.data, q.ctypes.data,
+                                         k.ctypes.data, v.ctypes.data, n, rows.ctypes.data,
+                                         o.ctypes.data, lse.ctypes.data)
     if err:
         raise MemoryError("oracle_attn_rows: allocation failed")
     return o, lse

@@ -348,12 +348,14 @@ int oracle_attn(const oracle_desc* d, const int64_t* prefix,
 /*
  * Selected rows only, for spot checks of large problems: rows[3*r + 0..2] =
  * (b, h, i) with i the position inside sequence b. o_rows is [nrows, D].
+ * The bias, when alibi_kind is set, is oracle_attn_alibi's.
  */
-int oracle_attn_rows(const oracle_desc* d, const int64_t* prefix,
-                     const int64_t* cu_q, const int64_t* cu_kv,
-                     const uint8_t* mask, const double* q, const double* k,
-                     const double* v, int64_t nrows, const int64_t* rows,
-                     double* o_rows, double* lse_rows) {
+int oracle_attn_rows_alibi(const oracle_desc* d, const int64_t* prefix,
+                           const int64_t* cu_q, const int64_t* cu_kv,
+                           const uint8_t* mask, int32_t alibi_kind,
+                           const double* slopes, const double* q, const double* k,
+                           const double* v, int64_t nrows, const int64_t* rows,
+                           double* o_rows, double* lse_rows) {
     int err = 0;
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t r = 0; r < nrows; ++r) {
@@ -362,22 +364,38 @@ int oracle_attn_rows(const oracle_desc* d, const int64_t* prefix,
         int64_t skv_alloc = s.skv > 0 ? s.skv : 1;
         uint8_t* vis = (uint8_t*)malloc((size_t)skv_alloc);
         double* scores = (double*)malloc(sizeof(double) * skv_alloc);
-        if (!vis || !scores) {
+        double* bias = (double*)malloc(sizeof(double) * skv_alloc);
+        if (!vis || !scores || !bias) {
             free(vis);
             free(scores);
+            free(bias);
 #pragma omp atomic write
             err = 1;
             continue;
         }
-        for (int64_t j = 0; j < s.skv; ++j)
+        for (int64_t j = 0; j < s.skv; ++j) {
             vis[j] = (uint8_t)oracle_visible(d, prefix, cu_q, cu_kv, mask, b,
                                              h, i, j);
-        attend_row(d, q, k, v, b, h, s, i, vis, NULL, scores, o_rows + r * d->D,
-                   lse_rows + r);
+            if (alibi_kind != OR_ALIBI_NONE)
+                bias[j] = slopes[h] * alibi_bias(alibi_kind, i, j, s.sq, s.skv);
+        }
+        attend_row(d, q, k, v, b, h, s, i, vis,
+                   alibi_kind != OR_ALIBI_NONE ? bias : NULL, scores,
+                   o_rows + r * d->D, lse_rows + r);
         free(vis);
         free(scores);
+        free(bias);
     }
     return err;
+}
+
+int oracle_attn_rows(const oracle_desc* d, const int64_t* prefix,
+                     const int64_t* cu_q, const int64_t* cu_kv,
+                     const uint8_t* mask, const double* q, const double* k,
+                     const double* v, int64_t nrows, const int64_t* rows,
+                     double* o_rows, double* lse_rows) {
+    return oracle_attn_rows_alibi(d, prefix, cu_q, cu_kv, mask, OR_ALIBI_NONE,
+                                  NULL, q, k, v, nrows, rows, o_rows, lse_rows);
 }
 
 /*

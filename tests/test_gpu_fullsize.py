@@ -10,7 +10,7 @@ import torch
 import masked_attention_fa_b200 as fa
 import oracle
 from oracle import Problem
-from masked_attention_fa_b200.workloads import make_inputs, named_workloads
+from masked_attention_fa_b200.workloads import alibi_slopes, make_inputs, named_workloads
 from gpu_helpers import TOL_LSE, TOL_MAX_O, TOL_MEAN_O
 
 pytestmark = pytest.mark.gpu
@@ -32,14 +32,22 @@ def _rows_of(sq, rng):
     return sorted({r for r in base + rnd if 0 <= r < sq})
 
 
+def _bias(w, slopes, h):
+    """The oracle's ALiBi arguments for head h of workload w (one head per
+    oracle problem)."""
+    return {} if w.alibi is None else {"alibi": w.alibi, "slopes": slopes[h:h + 1]}
+
+
 @pytest.mark.parametrize("name", ["leftup_causal_4k", "rightdown_band_2k_8k",
-                                  "varlen_rightdown_16seq", "prefix_8k"])
+                                  "varlen_rightdown_16seq", "prefix_8k", "alibi_causal_4k"])
 def test_named_workload_sampled_rows(name):
     w = named_workloads()[name]
     inp = make_inputs(w)
     attn = fa.MaskedAttention(w.layout, w.B, w.N, w.Sq, w.Skv, w.D, w.sparse_mode,
-                              w.pre_tokens, w.next_tokens, w.scale, w.mask_kind)
-    o, lse = attn(inp["q"].cuda(), inp["k"].cuda(), inp["v"].cuda(), **_arrays(w))
+                              w.pre_tokens, w.next_tokens, w.scale, w.mask_kind, w.alibi)
+    slopes = alibi_slopes(w.N) if w.alibi else None
+    o, lse = attn(inp["q"].cuda(), inp["k"].cuda(), inp["v"].cuda(), **_arrays(w),
+                  slopes=None if slopes is None else torch.tensor(slopes, device="cuda"))
     torch.cuda.synchronize()
     attn.sync_status()
     attn.close()
@@ -63,7 +71,8 @@ def test_named_workload_sampled_rows(name):
             sq = seq_lens[b][0]
             rows = _rows_of(sq, rng)
             if w.layout == "TND":
-                o_ref, l_ref = oracle.attention_rows(pb, qh, kh, vh, [(b, 0, i) for i in rows])
+                o_ref, l_ref = oracle.attention_rows(pb, qh, kh, vh, [(b, 0, i) for i in rows],
+                                                     **_bias(w, slopes, h))
                 got = o[[q0s[b] + i for i in rows], h]
                 gl = lse[h, [q0s[b] + i for i in rows]]
             else:
@@ -74,7 +83,8 @@ def test_named_workload_sampled_rows(name):
                               pre_tokens=w.pre_tokens, next_tokens=w.next_tokens,
                               scale=w.scale,
                               prefix=None if w.prefix is None else [w.prefix[b]])
-                o_ref, l_ref = oracle.attention_rows(pb1, qs, ks, vs, [(0, 0, i) for i in rows])
+                o_ref, l_ref = oracle.attention_rows(pb1, qs, ks, vs, [(0, 0, i) for i in rows],
+                                                     **_bias(w, slopes, h))
                 got = o[b, h, rows] if w.layout == "BNSD" else o[b, rows, h]
                 gl = lse[b, h, rows]
             errs.append(np.abs(got - o_ref))

@@ -418,3 +418,48 @@ def test_plan_items_reports_its_length_and_rejects_a_short_buffer():
     assert fa.STATUS[st] == "FA_ERR_NULLPTR"
     st = lib.fa_plan_items(ctypes.byref(desc), None, None, None, 4, None, ctypes.byref(n))
     assert fa.STATUS[st] == "FA_ERR_NULLPTR"
+
+
+def test_alibi_descriptor_checks():
+    """The descriptor's ALiBi variant: 0..3, and only without an attenMask."""
+    for kind in ("right", "sqrt", "left"):
+        assert _status(**BASE, sparse_mode=3, alibi=kind) == "FA_OK"
+        assert _status(**BASE, sparse_mode=0, alibi=kind) == "FA_OK"
+    assert _status(**BASE, sparse_mode=3, alibi=4) == "FA_ERR_PARAM_INVALID"
+    assert _status(**BASE, sparse_mode=3, alibi=-1) == "FA_ERR_PARAM_INVALID"
+    assert _status(**BASE, sparse_mode=1, mask_kind="SS", alibi="right") == "FA_ERR_UNSUPPORTED"
+    assert _status(**BASE, sparse_mode=0, mask_kind="BNSS", alibi="left") == "FA_ERR_UNSUPPORTED"
+
+
+def test_alibi_entry_points_validate_before_device_work():
+    """fa_fwd on an ALiBi handle, fa_fwd_alibi on a plain handle, missing or
+    unaligned slopes, and the entry points without slopes (allocation-free,
+    paged) are all refused on the host; the device pointers below are never
+    touched."""
+    import ctypes
+    lib = fa.load_library()
+    dev = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10002)
+    ali = fa.fa_create(fa.make_desc("BNSD", 1, 2, 64, 64, 64, 3, alibi="right"))
+    plain = fa.fa_create(fa.make_desc("BNSD", 1, 2, 64, 64, 64, 3))
+    tnd = fa.fa_create(fa.make_desc("TND", 1, 2, 1, 64, 64, 3, alibi="right"))
+    try:
+        st = lambda x: fa.STATUS[x]
+        assert st(lib.fa_fwd(ali, dev, dev, dev, None, None, None, None, dev, dev, None)) == \
+            "FA_ERR_PARAM_INVALID"
+        assert "fa_fwd_alibi" in fa.fa_last_error()
+        assert st(lib.fa_fwd_alibi(plain, dev, dev, dev, dev, None, None, None, dev, dev,
+                                   None)) == "FA_ERR_PARAM_INVALID"
+        assert st(lib.fa_fwd_alibi(ali, dev, dev, dev, None, None, None, None, dev, dev,
+                                   None)) == "FA_ERR_NULLPTR"
+        assert st(lib.fa_fwd_alibi(ali, dev, dev, dev, odd, None, None, None, dev, dev,
+                                   None)) == "FA_ERR_PARAM_INVALID"
+        d = fa.make_desc("BNSD", 1, 2, 64, 64, 64, 3, alibi="sqrt")
+        assert st(lib.fa_fwd_noalloc(ctypes.byref(d), dev, dev, dev, None, None, None, None,
+                                     dev, dev, None)) == "FA_ERR_UNSUPPORTED"
+        I64 = ctypes.c_int64 * 1
+        assert st(lib.fa_fwd_paged(tnd, dev, dev, dev, dev, 4, 16, 4, None, I64(1), I64(64),
+                                   dev, dev, None)) == "FA_ERR_UNSUPPORTED"
+    finally:
+        for h in (ali, plain, tnd):
+            fa.fa_destroy(h)

@@ -809,3 +809,16 @@ def test_alibi_with_zero_slopes_is_the_plain_forward():
     for kind in ("right", "sqrt", "left"):
         o, lse = oracle.attention(pb, q, k, v, alibi=kind, slopes=[0.0, 0.0])
         assert np.array_equal(o, o0) and np.array_equal(lse, l0)
+
+
+def test_alibi_rows_entry_matches_full_forward():
+    """The sampled-rows entry with a bias gives the full forward's rows."""
+    Sq, Skv, D, N = 9, 13, 8, 2
+    q, k, v = _rand((1, N, Sq, D), 95), _rand((1, N, Skv, D), 96), _rand((1, N, Skv, D), 97)
+    pb = Problem("BNSD", 1, N, Sq, Skv, D, sparse_mode=4, pre_tokens=5, next_tokens=2)
+    rows = [(0, h, i) for h in range(N) for i in range(Sq)]
+    for kind in ("right", "sqrt", "left"):
+        o, lse = oracle.attention(pb, q, k, v, alibi=kind, slopes=ALIBI_SLOPES)
+        orow, lrow = oracle.attention_rows(pb, q, k, v, rows, alibi=kind, slopes=ALIBI_SLOPES)
+        for r, (_, h, i) in enumerate(rows):
+            assert np.array_equal(orow[r], o[0, h, i]) and lrow[r] == lse[0, h, i]
