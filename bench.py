@@ -1,6 +1,7 @@
 """Benchmark of the B200 masked attention forward.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference] [--workload NAME]
+python bench.py --split [--workload split_rightdown_32k] ...   (under torchrun for N > 1)
 
 Prints ONE JSON line (rank 0). A step is one fa_fwd over the whole workload
 (every KV tile of every (sequence, head, query block)). The metric counts
@@ -13,6 +14,13 @@ scenarios (1.19 TFLOP of visible work per call). With --gpus N > 1 (under
 torchrun) every rank runs its own independent copy of the workload (the
 work shards by (batch, head, query block) with no exchange), so the value
 is the total over ranks divided by the slowest rank's time (weak scaling).
+
+--split runs the sparseMode page's multi-card scheme instead (sparseMode=7/8
+sections): the query tokens of one varlen rightDownCausal or leftUpCausal
+job are cut into N parts that balance the visible pairs (fa_split_queries),
+K/V stay whole, and rank r runs part r alone on its GPU: no collective in
+the forward. The value is the whole job's visible-pair FLOPs over the
+slowest rank's time (strong scaling: the job is fixed as N grows).
 
 Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events
 on the launching stream; a 256 MiB buffer (larger than the 126 MB L2) is
@@ -35,6 +43,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 DEFAULT_WORKLOAD = "prefix_8k"
+SPLIT_WORKLOAD = "split_rightdown_32k"
 METRIC = "masked-attention fwd TFLOP/s (visible pairs) and % of B200 BF16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -50,7 +59,12 @@ def parse():
                     help="budget of the oracle's bounded CPU sample")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    return ap.parse_args()
+    ap.add_argument("--split", action="store_true",
+                    help="run this rank's part of the query split of one varlen job")
+    args = ap.parse_args()
+    if args.split and args.workload == DEFAULT_WORKLOAD:
+        args.workload = SPLIT_WORKLOAD
+    return args
 
 
 def load_peaks():
@@ -342,6 +356,127 @@ def oracle_visible_pairs(w, mask_host=None):
     return total
 
 
+# ------------------------------------------------------------ query split
+
+def split_rank_part(w, world, rank):
+    """Part `rank` of `world` of the query split of TND job w (the sparseMode
+    page's multi-card scheme, fa_split_queries with cuts that balance the
+    visible pairs): its descriptor, cumulative arrays and token ranges."""
+    import masked_attention_fa_b200 as fa
+    if w.layout != "TND" or w.sparse_mode not in (2, 3):
+        raise ValueError("the query split takes a TND job in sparseMode 2 or 3")
+    d = fa.make_desc(w.layout, w.B, w.N, w.Sq, w.Skv, w.D, w.sparse_mode, w.pre_tokens,
+                     w.next_tokens, w.scale)
+    return fa.fa_split_queries(d, w.actual_seq_qlen, w.actual_seq_kvlen, world, rank)
+
+
+def split_part_inputs(inputs, part):
+    """The part's own q rows and the key/value rows it reads (views)."""
+    return {"q": inputs["q"][part["q_begin"]:part["q_end"]],
+            "k": inputs["k"][part["kv_begin"]:part["kv_end"]],
+            "v": inputs["v"][part["kv_begin"]:part["kv_end"]]}
+
+
+def split_step(part, inp, forward):
+    """One rank's forward of its part: forward(desc, q, k, v, cu_q, cu_kv)
+    -> (o, lse); None for a part without query tokens (nothing to run)."""
+    if part["q_end"] <= part["q_begin"]:
+        return None
+    return forward(part["desc"], inp["q"], inp["k"], inp["v"], part["actual_seq_qlen"],
+                   part["actual_seq_kvlen"])
+
+
+def run_split(args):
+    import torch
+    import torch.distributed as dist
+    import masked_attention_fa_b200 as fa
+    from masked_attention_fa_b200.workloads import named_workloads, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = named_workloads()[args.workload]
+    part = split_rank_part(w, world, rank)
+    inp = {x: t.to(dev) for x, t in split_part_inputs(make_inputs(w), part).items()}
+    pd = part["desc"]
+    attn = fa.MaskedAttention("TND", pd.B, pd.N, pd.Sq, pd.Skv, pd.D, pd.sparse_mode,
+                              pd.pre_tokens, pd.next_tokens, pd.scale)
+    oshape, lshape = attn.out_shapes()
+    o = torch.empty(oshape, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(lshape, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def cuda_forward(desc, q, k, v, cu_q, cu_kv):
+        return attn(q, k, v, actual_seq_qlen=cu_q, actual_seq_kvlen=cu_kv, out=o, lse=lse,
+                    stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        split_step(part, inp, cuda_forward)
+    torch.cuda.synchronize(dev)
+    attn.sync_status()
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        starts[i].record(stream)
+        split_step(part, inp, cuda_forward)
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    attn.sync_status()
+    ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    d = fa.make_desc(w.layout, w.B, w.N, w.Sq, w.Skv, w.D, w.sparse_mode, w.pre_tokens,
+                     w.next_tokens, w.scale)
+    pairs = fa.fa_visible_pairs(d, **workload_args(w))
+    my_pairs = 0
+    if part["q_end"] > part["q_begin"]:
+        my_pairs = fa.fa_visible_pairs(pd, actual_seq_qlen=part["actual_seq_qlen"],
+                                       actual_seq_kvlen=part["actual_seq_kvlen"])
+    flops = 4.0 * w.D * pairs
+    value = flops / (ms_max * 1e-3) / 1e12
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        peak = float(peaks["bf16_tflops"])
+        achieved = 4.0 * w.D * my_pairs / (ms * 1e-3) / 1e12
+        cfg = bench_config(w, pairs, world)
+        cfg["parallelism"] = f"query split x{world} (sparseMode=7/8 multi-card scheme)"
+        cfg["per_rank"] = (f"part {rank}: query tokens [{part['q_begin']}, {part['q_end']}), "
+                           f"keys [{part['kv_begin']}, {part['kv_end']}), sparse_mode "
+                           f"{pd.sparse_mode}")
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic", "config": cfg,
+                "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                             "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                             "peak_source": f"{peak_src} bf16_tflops (burst)",
+                             "kernel": "fa_fwd_sm100 (rank 0's part)", "kernel_ms": ms},
+                "cpu_baseline": None, "e2e": None, "gpu_launches": args.steps,
+                "clocks": clocks}
+        print(json.dumps(line))
+    attn.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def run_reference(args):
     """The oracle on the host cores, as the reference arm."""
     rank = int(os.environ.get("RANK", "0"))
@@ -385,6 +520,9 @@ def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.split:
+        run_split(args)
         return
 
     import torch

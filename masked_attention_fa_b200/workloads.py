@@ -226,6 +226,11 @@ def named_workloads() -> dict:
         # given as an explicit lower-triangular allMask (sparseMode 1)
         "allmask_causal_4k": Workload("allmask_causal_4k", "BNSD", 2, 16, 4096, 4096, 128, 1,
                                       seed=2, mask_kind="SS"),
+        # one long rightDownCausal sequence, the job the sparseMode=7/8
+        # sections cut across cards by query rows (bench.py --split)
+        "split_rightdown_32k": Workload("split_rightdown_32k", "TND", 1, 32, 32768, 32768, 128,
+                                        3, seed=7, actual_seq_qlen=[32768],
+                                        actual_seq_kvlen=[32768]),
         # decode: one query token per sequence against a long context held
         # in paged caches (blocks of 128 tokens in random order), mode 3
         "paged_decode_16k": Workload("paged_decode_16k", "TND", 16, 32, dq[-1], dkv[-1], 128, 3,
