@@ -162,7 +162,9 @@ fa_status_t fa_create(const fa_desc_t* desc, fa_handle_t* out);
  * Work distribution: items (sequence, head, 256 query rows) are sorted
  * longest first. A closed-form call whose list holds at least 8 items per
  * SM lets each CTA claim its next item from a counter in the workspace
- * while it loads its current one (the last CTA resets it); otherwise each
+ * while it loads its current one (the last CTA resets it), with the list
+ * grouped by (sequence, head) inside buckets of similar length so that the
+ * items in flight share K/V through L2 (see fa_plan_items); otherwise each
  * CTA takes a fixed share. Every output row is produced by one CTA either
  * way, so results do not depend on which CTA computed them.
  *
@@ -412,18 +414,24 @@ fa_status_t fa_plan_stats(const fa_desc_t* desc, const int64_t* prefix,
 
 /*
  * fa_plan_items — the work list of a closed-form call (no attenMask) in the
- * order the kernel takes it: longest first by the cost key 8 x (the longer
- * sub-tile's key tiles) + (the shorter's), ties in (sequence, block, head)
- * order, so items without a key tile come last. Item m is out[4m .. 4m+3] =
- * (sequence b, head h, block of 256 query rows, cost key). out: host
- * int32[4 * capacity], may be NULL when capacity is 0. *n_items receives the
- * list's length also when it exceeds capacity (then FA_ERR_SHAPE and out is
- * not written). Host only; dense-mask calls rebuild their list on the device
- * from the mask.
+ * order the kernel takes it on a device with num_sms SMs (148 on B200).
+ * The cost key of an item is 8 x (the longer sub-tile's key tiles) + (the
+ * shorter's). A list each CTA takes a fixed share of (fewer than 8 items
+ * per SM) is longest first, ties in (sequence, block, head) order. A list
+ * that is claimed at run time (at least 8 items per SM) is longest first by
+ * buckets of 16 key tiles (key / 128), and inside a bucket ordered by
+ * (sequence, head), then longest first, then block: the items in flight
+ * then share their K/V tiles through L2. Items without a key tile come last
+ * in both orders. Item m is out[4m .. 4m+3] = (sequence b, head h, block of
+ * 256 query rows, cost key). out: host int32[4 * capacity], may be NULL when
+ * capacity is 0. *n_items receives the list's length also when it exceeds
+ * capacity (then FA_ERR_SHAPE and out is not written). num_sms < 1 is
+ * FA_ERR_PARAM_INVALID. Host only; dense-mask calls rebuild their list on
+ * the device from the mask.
  */
 fa_status_t fa_plan_items(const fa_desc_t* desc, const int64_t* prefix,
                           const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
-                          int64_t capacity, int32_t* out, int64_t* n_items);
+                          int32_t num_sms, int64_t capacity, int32_t* out, int64_t* n_items);
 
 /* ---------------- query split across devices (host only) ---------------- */
 

@@ -104,7 +104,7 @@ def load_library():
     lib.fa_tile_class.restype = ctypes.c_int32
     lib.fa_plan_stats.argtypes = [dp, i64p, i64p, i64p, ctypes.c_int32, i64p]
     lib.fa_plan_stats.restype = st
-    lib.fa_plan_items.argtypes = [dp, i64p, i64p, i64p, ctypes.c_int64,
+    lib.fa_plan_items.argtypes = [dp, i64p, i64p, i64p, ctypes.c_int32, ctypes.c_int64,
                                   ctypes.POINTER(ctypes.c_int32), i64p]
     lib.fa_plan_items.restype = st
     lib.fa_fwd_noalloc.argtypes = [dp, P, P, P, P, i64p, i64p, i64p, P, P, P]
@@ -203,19 +203,20 @@ def fa_tile_class(desc, b, qt, kt, prefix=None, actual_seq_qlen=None, actual_seq
                                              int(b), int(qt), int(kt)))
 
 
-def fa_plan_items(desc, prefix=None, actual_seq_qlen=None, actual_seq_kvlen=None):
-    """The closed-form work list in the kernel's order: int32 array [n, 4] of
-    (sequence, head, 256-row block, cost key)."""
+def fa_plan_items(desc, prefix=None, actual_seq_qlen=None, actual_seq_kvlen=None, num_sms=148):
+    """The closed-form work list in the kernel's order on a device with
+    num_sms SMs: int32 array [n, 4] of (sequence, head, 256-row block, cost
+    key)."""
     import numpy as np
     a = _Arrays(prefix, actual_seq_qlen, actual_seq_kvlen)
     n = ctypes.c_int64(0)
     lib = load_library()
-    st = lib.fa_plan_items(ctypes.byref(desc), *a.ptrs(), 0, None, ctypes.byref(n))
+    st = lib.fa_plan_items(ctypes.byref(desc), *a.ptrs(), int(num_sms), 0, None, ctypes.byref(n))
     if n.value == 0:
         _check(st)
         return np.zeros((0, 4), dtype=np.int32)
     out = np.zeros((n.value, 4), dtype=np.int32)
-    _check(lib.fa_plan_items(ctypes.byref(desc), *a.ptrs(), n.value,
+    _check(lib.fa_plan_items(ctypes.byref(desc), *a.ptrs(), int(num_sms), n.value,
                              out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), ctypes.byref(n)))
     return out
 

@@ -184,6 +184,9 @@ fa_status_t refresh_plan(fa_handle_t h, const int64_t* prefix, const int64_t* cu
   std::vector<SeqRec> recs = decode_geometry(&h->desc, prefix, cu_q, cu_kv, has_mask);
   std::vector<WorkItem> items = build_items(&h->desc, recs);
   if (items.size() > (size_t)0x7fffffff) return fail(FA_ERR_UNSUPPORTED, "too many work items");
+  // Claimed lists (closed form only) take the L2-locality order.
+  if (!has_mask && claims_items((int64_t)items.size(), h->num_sms))
+    order_work_list(items.data(), items.data() + items.size(), true);
   const size_t seq_bytes = recs.size() * sizeof(SeqRec);
   const size_t item_bytes = items.size() * sizeof(WorkItem);
   const int64_t planes = mask_planes(&h->desc, has_mask);
@@ -408,8 +411,7 @@ fa_status_t forward(fa_handle_t h, const void* q, const void* k, const void* v,
   p.n_items = h->n_items;
   // Closed-form lists (descending lpt_key: items without a key tile last)
   // with many items per CTA are claimed at run time.
-  if (!has_mask && (int64_t)h->n_items >= (int64_t)kClaimMinItemsPerCta * h->num_sms &&
-      h->n_items < 0x7fff0000) {
+  if (!has_mask && claims_items(h->n_items, h->num_sms)) {
     p.claim = reinterpret_cast<unsigned int*>(ws + kClaimOffset);
     p.claim_done = reinterpret_cast<unsigned int*>(ws + kClaimOffset + 64);
   }

@@ -256,14 +256,13 @@ extern "C" fa_status_t fa_fwd_noalloc(const fa_desc_t* desc, const void* q, cons
       for (int64_t h = 0; h < desc->N; ++h) items[n++] = WorkItem{(int32_t)b, (int32_t)h, qb, cost};
     }
   }
-  // Descending cost, ties in generation order (b, block, head): the same
-  // order a stable sort by cost gives, without a temporary buffer.
-  std::sort(items, items + n, [](const WorkItem& a, const WorkItem& c) {
-    if (a.cost != c.cost) return a.cost > c.cost;
-    if (a.b != c.b) return a.b < c.b;
-    if (a.qblk != c.qblk) return a.qblk < c.qblk;
-    return a.h < c.h;
-  });
+  // The handle path's order (in place, no temporary buffer): strict longest
+  // first, or the L2-locality order for a list that is claimed at run time
+  // (a closed-form list with room for its ranges, see below).
+  const size_t tr_need = round256(need) + n * 2 * sizeof(TileRange);
+  const bool claimed = !has_mask && tr_need <= kNoAllocScratchBytes &&
+                       claims_items((int64_t)n, slot->num_sms);
+  order_work_list(items, items + n, claimed);
 
   unsigned char* dscr = static_cast<unsigned char*>(slot->scratch);
   e = cudaMemsetAsync(dscr, 0, kNoAllocHeaderBytes, stream);  // error word = 0
@@ -320,7 +319,7 @@ extern "C" fa_status_t fa_fwd_noalloc(const fa_desc_t* desc, const void* q, cons
       p.item_tr = reinterpret_cast<const TileRange*>(dscr + tr_off);
       // Claimed work as in fa_fwd; the counters sit in the header, which
       // was zeroed above.
-      if (n >= (size_t)kClaimMinItemsPerCta * (size_t)slot->num_sms && n < 0x7fff0000u) {
+      if (claimed) {
         p.claim = reinterpret_cast<unsigned int*>(dscr + 128);
         p.claim_done = reinterpret_cast<unsigned int*>(dscr + 192);
       }

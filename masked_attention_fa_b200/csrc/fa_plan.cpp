@@ -7,6 +7,7 @@
 //   sparseMode=7 and sparseMode=8 (the band-piece conditions and Sq <= Skv
 //   for the other batches).
 #include "fa_plan.h"
+#include "fa_kernel.h"
 
 #include <algorithm>
 #include <cmath>
@@ -270,9 +271,37 @@ std::vector<WorkItem> build_items(const fa_desc_t* d, const std::vector<SeqRec>&
         items.push_back(WorkItem{(int32_t)b, (int32_t)h, qb, cost});
     }
   }
-  std::stable_sort(items.begin(), items.end(),
-                   [](const WorkItem& a, const WorkItem& c) { return a.cost > c.cost; });
+  order_work_list(items.data(), items.data() + items.size(), false);
   return items;
+}
+
+bool claims_items(int64_t n_items, int num_sms) {
+  return n_items >= (int64_t)kClaimMinItemsPerCta * num_sms && n_items < 0x7fff0000;
+}
+
+void order_work_list(WorkItem* first, WorkItem* last, bool locality) {
+  // The cost key is 8 x (the longer sub-tile's key tiles) + (the
+  // shorter's); 8 x kLocalityTiles of it make one bucket.
+  constexpr int32_t kBucket = 8 * kLocalityTiles;
+  if (!locality) {
+    std::sort(first, last, [](const WorkItem& a, const WorkItem& c) {
+      if (a.cost != c.cost) return a.cost > c.cost;
+      if (a.b != c.b) return a.b < c.b;
+      if (a.qblk != c.qblk) return a.qblk < c.qblk;
+      return a.h < c.h;
+    });
+    return;
+  }
+  std::sort(first, last, [](const WorkItem& a, const WorkItem& c) {
+    const bool ea = a.cost == 0, ec = c.cost == 0;  // no key tile: last
+    if (ea != ec) return ec;
+    const int32_t ba = a.cost / kBucket, bc = c.cost / kBucket;
+    if (ba != bc) return ba > bc;
+    if (a.b != c.b) return a.b < c.b;
+    if (a.h != c.h) return a.h < c.h;
+    if (a.cost != c.cost) return a.cost > c.cost;
+    return a.qblk < c.qblk;
+  });
 }
 
 fa_status_t validate_paged(const fa_desc_t* d, const int64_t* prefix, const int64_t* cu_q,
@@ -609,15 +638,18 @@ fa_status_t fa_plan_stats(const fa_desc_t* desc, const int64_t* prefix,
 
 fa_status_t fa_plan_items(const fa_desc_t* desc, const int64_t* prefix,
                           const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
-                          int64_t capacity, int32_t* out, int64_t* n_items) {
+                          int32_t num_sms, int64_t capacity, int32_t* out, int64_t* n_items) {
   clear_error();
   if (!n_items) return fail(FA_ERR_NULLPTR, "n_items is NULL");
   if (capacity < 0) return fail(FA_ERR_PARAM_INVALID, "capacity %lld < 0", (long long)capacity);
   if (capacity > 0 && !out) return fail(FA_ERR_NULLPTR, "out is NULL");
+  if (num_sms < 1) return fail(FA_ERR_PARAM_INVALID, "num_sms %d < 1", num_sms);
   fa_status_t st = validate_call(desc, prefix, actual_seq_qlen, actual_seq_kvlen, 0);
   if (st != FA_OK) return st;
   auto recs = decode_geometry(desc, prefix, actual_seq_qlen, actual_seq_kvlen, 0);
   auto items = build_items(desc, recs);
+  if (claims_items((int64_t)items.size(), num_sms))
+    order_work_list(items.data(), items.data() + items.size(), true);
   *n_items = (int64_t)items.size();
   if ((int64_t)items.size() > capacity)
     return fail(FA_ERR_SHAPE, "the work list has %zu items, capacity %lld", items.size(),

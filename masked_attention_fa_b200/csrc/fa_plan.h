@@ -30,6 +30,23 @@ inline int32_t lpt_key(const TileRange& a, const TileRange& b) {
   return ta > tb ? 8 * ta + tb : 8 * tb + ta;
 }
 std::vector<WorkItem> build_items(const fa_desc_t* d, const std::vector<SeqRec>& recs);
+// Whether a closed-form list of n_items is claimed at run time on num_sms
+// SMs (the kernel's claiming instance, at least kClaimMinItemsPerCta items
+// per SM).
+bool claims_items(int64_t n_items, int num_sms);
+// Orders a closed-form work list in place, allocating nothing. Strict
+// longest first (ties in (sequence, block, head) order) for lists each CTA
+// takes a fixed share of; for claimed lists (locality = true), longest
+// first by buckets of kLocalityTiles key tiles, and inside a bucket the
+// items of one (sequence, head) together, so that the CTAs claiming
+// consecutive items read the same K/V tiles at about the same time and
+// share them through L2 (with strict order the ~148 items in flight come
+// from as many (sequence, head) pairs, whose K/V outgrow L2 and are read
+// from DRAM by every item: 3.7x the algorithmic bytes on a causal-prefix
+// problem of 8k tokens, 4.5x on 16 varlen sequences). Items without a key
+// tile come last either way (claiming relies on it).
+constexpr int32_t kLocalityTiles = 16;
+void order_work_list(WorkItem* first, WorkItem* last, bool locality);
 int64_t visible_pairs(const fa_desc_t* d, const std::vector<SeqRec>& recs);
 int32_t tile_class(const SeqRec& s, int64_t qt, int64_t kt);
 

@@ -412,11 +412,11 @@ def test_plan_items_reports_its_length_and_rejects_a_short_buffer():
     lib = fa.load_library()
     n = ctypes.c_int64(-1)
     buf = (ctypes.c_int32 * 8)()
-    st = lib.fa_plan_items(ctypes.byref(desc), None, None, None, 2, buf, ctypes.byref(n))
+    st = lib.fa_plan_items(ctypes.byref(desc), None, None, None, 148, 2, buf, ctypes.byref(n))
     assert fa.STATUS[st] == "FA_ERR_SHAPE" and n.value == 6   # 3 blocks x 2 heads
-    st = lib.fa_plan_items(ctypes.byref(desc), None, None, None, 0, None, None)
+    st = lib.fa_plan_items(ctypes.byref(desc), None, None, None, 148, 0, None, None)
     assert fa.STATUS[st] == "FA_ERR_NULLPTR"
-    st = lib.fa_plan_items(ctypes.byref(desc), None, None, None, 4, None, ctypes.byref(n))
+    st = lib.fa_plan_items(ctypes.byref(desc), None, None, None, 148, 4, None, ctypes.byref(n))
     assert fa.STATUS[st] == "FA_ERR_NULLPTR"
 
 
@@ -463,3 +463,55 @@ def test_alibi_entry_points_validate_before_device_work():
     finally:
         for h in (ali, plain, tnd):
             fa.fa_destroy(h)
+
+
+def _expected_keys(c, prefix, cu_q, cu_kv):
+    """Each item's cost key from the oracle's block ranges."""
+    pb = Problem(**c, prefix=prefix, actual_seq_qlen=cu_q, actual_seq_kvlen=cu_kv)
+    expected = {}
+    for b in range(c["B"]):
+        sq = pb.seq(b)[2]
+        if sq <= 0:
+            continue
+        r = oracle.tile_ranges(oracle.tile_classes(pb, b))
+        tiles = [int(r[qt, 1] - r[qt, 0]) if qt < len(r) else 0 for qt in range(len(r) + 1)]
+        for qb in range((sq + 255) // 256):
+            t0, t1 = tiles[2 * qb], tiles[2 * qb + 1]
+            for h in range(c["N"]):
+                expected[(b, h, qb)] = 8 * max(t0, t1) + min(t0, t1)
+    return expected
+
+
+@pytest.mark.parametrize("num_sms", [148, 8])
+def test_claimed_list_order_groups_sequence_and_head_inside_length_buckets(num_sms):
+    """A list with at least 8 items per SM (claimed at run time) is ordered for
+    L2 locality: items without a key tile last, then buckets of 16 key tiles
+    (key // 128) longest first, inside a bucket (sequence, head) ascending,
+    then the key descending, then the block; every item once with the oracle's
+    key. With fewer items per SM the same call gives the strict order."""
+    g = np.random.default_rng(9)
+    qlen = g.integers(0, 1500, size=40).tolist()
+    kvlen = [q + int(g.integers(0, 300)) for q in qlen]
+    kvlen[3] = 0                                        # a sequence without keys
+    cu_q, cu_kv = np.cumsum(qlen).tolist(), np.cumsum(kvlen).tolist()
+    c = dict(layout="TND", B=40, N=6, Sq=cu_q[-1], Skv=cu_kv[-1], D=64, sparse_mode=3)
+    desc = fa.make_desc(**c)
+    items = fa.fa_plan_items(desc, actual_seq_qlen=cu_q, actual_seq_kvlen=cu_kv, num_sms=num_sms)
+    got = {(int(b), int(h), int(qb)): int(key) for b, h, qb, key in items}
+    assert len(got) == len(items) and got == _expected_keys(c, None, cu_q, cu_kv)
+    keys = items[:, 3]
+    claimed = len(items) >= fa.CLAIM_MIN_ITEMS_PER_CTA * num_sms
+    assert claimed == (num_sms == 8)
+    if not claimed:
+        assert np.all(keys[:-1] >= keys[1:])
+        return
+    zero = keys == 0
+    assert zero.any() and not np.any(zero[:-1] & ~zero[1:]), "items without a key tile last"
+    k = keys[~zero]
+    it = items[~zero]
+    buckets = k // 128
+    assert np.all(buckets[:-1] >= buckets[1:])
+    for m in range(len(it) - 1):
+        if buckets[m] == buckets[m + 1]:
+            a, z = it[m], it[m + 1]
+            assert (a[0], a[1], -a[3], a[2]) < (z[0], z[1], -z[3], z[2])
