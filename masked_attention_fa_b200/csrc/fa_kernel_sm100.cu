@@ -44,6 +44,39 @@
 namespace fa {
 namespace dev {
 
+// Trace builds only (-DFA_TRACE, made by masked_attention_fa_b200/trace.py):
+// clock64 stamps of one CTA at the points where the roles wait and hand
+// work over, per key tile; compiled out of the library itself.
+#ifdef FA_TRACE
+constexpr int kTraceN = 1024;
+__device__ unsigned long long g_fa_trace[8][8][kTraceN];   // [row][event][tile]
+__device__ unsigned long long g_fa_wtrace[8][4][kTraceN];  // [softmax warp][event][turn]
+__device__ int g_fa_trace_cta;
+__device__ __forceinline__ unsigned long long trace_clock() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
+  return t;
+}
+#define FA_STAMP(r, e, n)                                                          \
+  do {                                                                             \
+    if ((int)blockIdx.x == g_fa_trace_cta && (uint32_t)(n) < (uint32_t)kTraceN)  \
+      g_fa_trace[r][e][n] = trace_clock();                                         \
+  } while (0)
+#define FA_WSTAMP(e, n)                                                                 \
+  do {                                                                                  \
+    if ((threadIdx.x & 31) == 0 && (int)blockIdx.x == g_fa_trace_cta &&                \
+        (uint32_t)(n) < (uint32_t)kTraceN)                                              \
+      g_fa_wtrace[threadIdx.x >> 5][e][n] = trace_clock();                             \
+  } while (0)
+#else
+#define FA_STAMP(r, e, n) \
+  do {                    \
+  } while (0)
+#define FA_WSTAMP(e, n) \
+  do {                  \
+  } while (0)
+#endif
+
 constexpr int kThreads = 512;
 constexpr int kWarpMma = 12;
 constexpr int kWarpLoad = 13;
@@ -538,9 +571,11 @@ __device__ void load_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint8_t
   };
   auto load_kv = [&](const CUtensorMap* tm, int row, int h, int bc) -> bool {
     const uint32_t st = ring % NS;
+    FA_STAMP(6, 0, ring);
     if (ring >= (uint32_t)NS &&
         !wait_bounded(&ctl->kv_empty[st], ((ring / NS) - 1) & 1u, w, kSiteKvEmpty))
       return false;
+    FA_STAMP(6, 1, ring);
     mbar_expect_tx(&ctl->kv_full[st], C::kTileBytes);
 #pragma unroll
     for (int c = 0; c < C::kChunks; ++c)
@@ -752,6 +787,7 @@ __device__ void qk_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
     bool q_ready[2] = {false, false};
     for (int t = cur.lo[2]; t < cur.hi[2] && ok; ++t, ++g) {
       const uint32_t r = ring_k(g);
+      FA_STAMP(2, 0, g);
       if (!wait_bounded(&ctl->kv_full[r % NS], (r / NS) & 1u, w, kSiteKvFull)) {
         ok = false;
         break;
@@ -767,12 +803,14 @@ __device__ void qk_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
           ++nq[s];
           q_ready[s] = true;
         }
+        FA_STAMP(2, 2 + s, g);
         if (n_qk[s] > 0 &&
             !wait_bounded(&ctl->s_free[s], (n_qk[s] - 1) & 1u, w, kSiteSFree)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        FA_STAMP(2, 4 + s, g);
         issue_qk<D>(tmem, sQ, sKV, s, r % NS);
         mma_commit(&ctl->s_full[s]);
         ++n_qk[s];
@@ -826,6 +864,7 @@ __device__ void pv_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
         }
       }
       const uint32_t r = ring_v(g, !have_next && last_t);
+      FA_STAMP(3, 0, g);
       if (!wait_bounded(&ctl->kv_full[r % NS], (r / NS) & 1u, w, kSiteKvFull)) {
         ok = false;
         break;
@@ -833,6 +872,7 @@ __device__ void pv_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
 #pragma unroll
       for (int s = 0; s < 2; ++s) {
         if (!act(cur, s, t)) continue;
+        FA_STAMP(3, 2 + s, g);
         if (!wait_bounded(&ctl->p_full[s], p_count[s] & 1u, w, kSitePFull)) {
           ok = false;
           break;
@@ -849,6 +889,7 @@ __device__ void pv_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
           ++n_act[s];
         }
         tc_fence_after();
+        FA_STAMP(3, 4 + s, g);
         issue_pv<D>(tmem, sP, sKV, s, r % NS, !first[s]);
         first[s] = false;
         mma_commit(&ctl->o_pv[s]);
@@ -1030,6 +1071,7 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
     if constexpr (kClaim) idx = idx_take_warp(ctl, k, w);
     else idx = item_index(k);
     if (idx >= p.n_items) break;
+    if (threadIdx.x == 0) FA_STAMP(5, 0, k);
     const WorkItem it = p.items[idx];
     const SeqRec sr = p.seqs[it.b];
     // The next item's record is read at the item boundary, on the critical
@@ -1091,6 +1133,7 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
         continue;
       }
       prefetch_mask(t + 1);
+      if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 0, turn - 1);
       if (!wait_warp(&ctl->s_full[sub], s_count & 1u, w, kSiteSFull)) {
         ok = false;
         break;
@@ -1135,9 +1178,11 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
           }
         }
       }
+      if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 1, turn - 1);
       tc_fence_after();
       float x[128];
       load_scores(tS, x, partial, c_lo, c_hi, mrow != nullptr, mbits);
+      if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 2, turn - 1);
       // S_s is in registers: the next QK of this sub-tile may overwrite it.
       tc_fence_before();
       mbar_arrive(&ctl->s_free[sub]);
@@ -1154,10 +1199,14 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
         m_used = m_new;
       }
       float zero = 0.f;
+      if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 3, turn - 1);
+      FA_WSTAMP(2, turn - 1);
       if (!first_turn && !turn_wait(sub, m_new, zero, w.abort_flag)) {
         ok = false;
         break;
       }
+      if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 4, turn - 1);
+      FA_WSTAMP(0, turn - 1);
       const float ref = ((m_used == -INFINITY) ? 0.f : m_used) + zero;
       const float mul = kAlibi ? 1.f : scale_log2;
       const uint64_t m2 = pack_f32x2(mul, mul);
@@ -1185,6 +1234,8 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
         exp_pack_part<false, kTokenCol, 128>(x, m2, c2, acc, pk);
       }
       l += sum_acc(acc);
+      if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 5, turn - 1);
+      FA_WSTAMP(1, turn - 1);
       if (pv_count > 0) {
         // The previous PV of this sub-tile must be done: it still reads the
         // P buffer, and O_s must hold it before it is rescaled.
@@ -1193,6 +1244,7 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
           break;
         }
         tc_fence_after();
+        if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 6, turn - 1);
         // Not on the item's first tile: the first PV of an item overwrites O_s.
         if (t > tr.lo && __any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
@@ -1215,6 +1267,8 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&ctl->p_full[sub]);
+      if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 7, turn - 1);
+      FA_WSTAMP(3, turn - 1);
       ++pv_count;
     }
     if (!ok) break;
@@ -1263,6 +1317,7 @@ __device__ void epilogue_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl,
       const TileRange tr = sub_range<kOcc>(p, idx, it, sr, sub);
       const int i = (int)(r0 + row);
       const bool row_valid = i < sr.sq;
+      if (threadIdx.x == 256) FA_STAMP(4, 3 * sub, k);
       if (!wait_warp(&ctl->epi_full[sub], k & 1u, w, kSiteEpi)) return;
       const float inv_l = inv_l_sm[sub * kTileM + row];
       mbar_arrive(&ctl->stat_free[sub]);
@@ -1272,8 +1327,10 @@ __device__ void epilogue_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl,
         const uint32_t npv = (sub ? n_pv1 : n_pv0) + (uint32_t)(tr.hi - tr.lo);
         if (sub) n_pv1 = npv;
         else n_pv0 = npv;
+        if (threadIdx.x == 256) FA_STAMP(4, 1 + 3 * sub, k);
         if (!wait_warp(&ctl->o_pv[sub], (npv - 1) & 1u, w, kSiteOPv)) return;
         tc_fence_after();
+        if (threadIdx.x == 256) FA_STAMP(4, 2 + 3 * sub, k);
         const uint32_t tO = tmem + lane_bits + C::col_o(sub);
 #pragma unroll 1
         for (int ch = 0; ch < D / 32; ++ch) {
@@ -1317,6 +1374,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100(const __grid_constan
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  if (threadIdx.x == 0) FA_STAMP(7, 0, 0);
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ctl->q_full[s], 1);
@@ -1494,3 +1552,23 @@ cudaError_t launch_fwd(int D, const FwdParams& p, int grid, cudaStream_t stream,
 }
 
 }  // namespace fa
+
+#ifdef FA_TRACE
+// Trace builds only: choose the traced CTA, clear and read the stamps.
+extern "C" int fa_trace_set_cta(int cta) {
+  return (int)cudaMemcpyToSymbol(fa::dev::g_fa_trace_cta, &cta, sizeof(cta));
+}
+extern "C" int fa_trace_clear(void) {
+  static unsigned long long zero[8 * 8 * fa::dev::kTraceN];
+  cudaError_t e = cudaMemcpyToSymbol(fa::dev::g_fa_trace, zero, sizeof(zero));
+  if (e == cudaSuccess)
+    e = cudaMemcpyToSymbol(fa::dev::g_fa_wtrace, zero, sizeof(fa::dev::g_fa_wtrace));
+  return (int)e;
+}
+extern "C" int fa_trace_read(void* tiles, void* warps) {
+  cudaError_t e = cudaMemcpyFromSymbol(tiles, fa::dev::g_fa_trace, sizeof(fa::dev::g_fa_trace));
+  if (e == cudaSuccess)
+    e = cudaMemcpyFromSymbol(warps, fa::dev::g_fa_wtrace, sizeof(fa::dev::g_fa_wtrace));
+  return (int)e;
+}
+#endif
