@@ -44,14 +44,14 @@
 namespace fa {
 namespace dev {
 
-// Trace builds only (-DFA_TRACE, made by masked_attention_fa_b200/trace.py):
-// clock64 stamps of one CTA at the points where the roles wait and hand
-// work over, per key tile; compiled out of the library itself.
+// Trace builds only (-DFA_TRACE=<cta>, made by masked_attention_fa_b200/
+// trace.py): clock64 stamps of CTA <cta> at the points where the roles wait
+// and hand work over, per key tile; compiled out of the library itself. The
+// traced CTA is a compile-time constant so a stamp costs no load.
 #ifdef FA_TRACE
 constexpr int kTraceN = 1024;
 __device__ unsigned long long g_fa_trace[8][8][kTraceN];   // [row][event][tile]
 __device__ unsigned long long g_fa_wtrace[8][4][kTraceN];  // [softmax warp][event][turn]
-__device__ int g_fa_trace_cta;
 __device__ __forceinline__ unsigned long long trace_clock() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
@@ -59,12 +59,12 @@ __device__ __forceinline__ unsigned long long trace_clock() {
 }
 #define FA_STAMP(r, e, n)                                                          \
   do {                                                                             \
-    if ((int)blockIdx.x == g_fa_trace_cta && (uint32_t)(n) < (uint32_t)kTraceN)  \
+    if ((int)blockIdx.x == (FA_TRACE) && (uint32_t)(n) < (uint32_t)kTraceN)      \
       g_fa_trace[r][e][n] = trace_clock();                                         \
   } while (0)
 #define FA_WSTAMP(e, n)                                                                 \
   do {                                                                                  \
-    if ((threadIdx.x & 31) == 0 && (int)blockIdx.x == g_fa_trace_cta &&                \
+    if ((threadIdx.x & 31) == 0 && (int)blockIdx.x == (FA_TRACE) &&                    \
         (uint32_t)(n) < (uint32_t)kTraceN)                                              \
       g_fa_wtrace[threadIdx.x >> 5][e][n] = trace_clock();                             \
   } while (0)
@@ -1554,10 +1554,8 @@ cudaError_t launch_fwd(int D, const FwdParams& p, int grid, cudaStream_t stream,
 }  // namespace fa
 
 #ifdef FA_TRACE
-// Trace builds only: choose the traced CTA, clear and read the stamps.
-extern "C" int fa_trace_set_cta(int cta) {
-  return (int)cudaMemcpyToSymbol(fa::dev::g_fa_trace_cta, &cta, sizeof(cta));
-}
+// Trace builds only: the traced CTA, and clearing and reading the stamps.
+extern "C" int fa_trace_cta(void) { return FA_TRACE; }
 extern "C" int fa_trace_clear(void) {
   static unsigned long long zero[8 * 8 * fa::dev::kTraceN];
   cudaError_t e = cudaMemcpyToSymbol(fa::dev::g_fa_trace, zero, sizeof(zero));

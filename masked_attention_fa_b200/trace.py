@@ -3,9 +3,9 @@
     python -m masked_attention_fa_b200.trace --workload prefix_8k [--cta 0] [--out FILE.npz]
     python -m masked_attention_fa_b200.trace --exp-probe
 
-Builds a second copy of the library with -DFA_TRACE (in
+Builds a second copy of the library with -DFA_TRACE=<cta> (in
 masked_attention_fa_b200/_trace/, separate from the library itself, whose
-kernel has no trace code), runs the named workload three times, then once
+kernel has no trace code; one copy per traced CTA), runs the named workload three times, then once
 more with the traced CTA's clock64 stamps recorded, and prints:
 
   - per softmax warpgroup and key tile, the median cycles of each phase:
@@ -38,24 +38,24 @@ import numpy as np
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 TRACE_DIR = os.path.join(HERE, "_trace")
-TRACE_LIB = os.path.join(TRACE_DIR, "libfa_b200_trace.so")
 N_TRACE = 1024
 
 
-def build_trace() -> str:
-    """Compile the library's sources with -DFA_TRACE into TRACE_LIB."""
+def build_trace(cta: int) -> str:
+    """Compile the library's sources with -DFA_TRACE=<cta>; returns the path."""
     from masked_attention_fa_b200 import build as b
     os.makedirs(TRACE_DIR, exist_ok=True)
+    lib = os.path.join(TRACE_DIR, f"libfa_b200_trace{int(cta)}.so")
     newest = max(os.path.getmtime(f) for f in b._inputs())
-    if os.path.exists(TRACE_LIB) and os.path.getmtime(TRACE_LIB) > newest:
-        return TRACE_LIB
-    cmd = [b.nvcc()] + b.NVCC_FLAGS + ["-DFA_TRACE", "-I" + os.path.join(ROOT, "include"),
-                                        "-o", TRACE_LIB] + b.sources()
+    if os.path.exists(lib) and os.path.getmtime(lib) > newest:
+        return lib
+    cmd = [b.nvcc()] + b.NVCC_FLAGS + [f"-DFA_TRACE={int(cta)}",
+                                        "-I" + os.path.join(ROOT, "include"), "-o", lib] + b.sources()
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
         raise RuntimeError("nvcc failed building the trace library")
-    return TRACE_LIB
+    return lib
 
 
 def record(workload: str, cta: int):
@@ -63,9 +63,8 @@ def record(workload: str, cta: int):
     arrays [8, 8, N] and [8, 4, N] (0 = not stamped)."""
     import torch
     import masked_attention_fa_b200 as fa
-    fa.LIB_PATH = build_trace()
+    fa.LIB_PATH = build_trace(cta)
     lib = fa.load_library()
-    lib.fa_trace_set_cta.argtypes = [ctypes.c_int]
     lib.fa_trace_read.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     sys.path.insert(0, ROOT)
     import bench
@@ -82,7 +81,7 @@ def record(workload: str, cta: int):
     for _ in range(3):
         attn(q, k, v, out=o, lse=l, slopes=slopes, **arrays)
     torch.cuda.synchronize()
-    if lib.fa_trace_set_cta(int(cta)) != 0 or lib.fa_trace_clear() != 0:
+    if lib.fa_trace_cta() != int(cta) or lib.fa_trace_clear() != 0:
         raise RuntimeError("trace set-up failed")
     flush.fill_(1.0)  # cold L2, as in the bench
     torch.cuda.synchronize()
