@@ -753,7 +753,9 @@ def main():
                 "config": bench_config(w, pairs, world),
                 "frac_of_peak": value / world / peak,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": args.steps * (4 if dense else (2 if paged else 1)),
+                # per step: the pre-pass, the work-list rebuild and the attention
+                # (dense mask); the partial and merge kernels (paged); else one
+                "gpu_launches": args.steps * (3 if dense else (2 if paged else 1)),
                 "clocks": clocks,
                 "ms_min": min(times_ms), "ms_median": statistics.median(times_ms)}
         if prepass_line is not None:

@@ -515,3 +515,17 @@ def test_claimed_list_order_groups_sequence_and_head_inside_length_buckets(num_s
         if buckets[m] == buckets[m + 1]:
             a, z = it[m], it[m + 1]
             assert (a[0], a[1], -a[3], a[2]) < (z[0], z[1], -z[3], z[2])
+
+
+def test_trace_build_compiles_and_exports_its_accessors():
+    """The per-cycle trace build (-DFA_TRACE=<cta>, masked_attention_fa_b200/trace.py) still
+    compiles from the library's sources and exports the traced CTA and the stamp accessors;
+    the library itself exports none of them (its kernel has no trace code)."""
+    import ctypes
+    from masked_attention_fa_b200 import trace
+    lib = ctypes.CDLL(trace.build_trace(3))
+    for name in ("fa_trace_cta", "fa_trace_clear", "fa_trace_read", "fa_create", "fa_fwd"):
+        assert hasattr(lib, name), name
+    assert lib.fa_trace_cta() == 3
+    prod = fa.load_library()
+    assert not hasattr(prod, "fa_trace_read")
