@@ -16,6 +16,8 @@ more with the traced CTA's clock64 stamps recorded, and prints:
     last exponential of one warpgroup to the first of the other);
   - the MMA issuers' waits for K/V, for S to be read and for P, and the TMA
     thread's waits for a free ring slot;
+  - per softmax warpgroup, the item boundary: reading the next item's
+    records and ranges, and handing the finished item's 1/l and lse over;
   - the traced CTA's item starts and its span.
 
 Stamps are clock64 of the SM running the CTA; with --out the raw arrays are
@@ -146,6 +148,19 @@ def summarize(tiles, warps) -> str:
     m = (tma[0] > 0) & (tma[1] > 0)
     out.append(f"TMA thread: free-slot wait median {_med((tma[1] - tma[0])[m])} over {m.sum()} "
                f"loads")
+    out.append("")
+    out.append("item boundary per softmax warpgroup (median cycles over the items after the "
+               "first): index -> item record -> sequence record -> tile ranges -> row set-up; "
+               "last turn -> 1/l slot free -> lse stored -> next index")
+    for s, r in ((0, 5), (1, 7)):
+        e = tiles[r]
+        ks = [k for k in np.nonzero(e[0] > 0)[0] if k > 0]
+        seg = [_med([e[j + 1, k] - e[j, k] for k in ks if e[j + 1, k] > 0]) for j in range(4)]
+        end = [_med([e[j + 1, k] - e[j, k] for k in ks if e[j, k] > 0 and e[j + 1, k] > 0])
+               for j in (5, 6)]
+        nxt = _med([e[0, k] - e[7, k - 1] for k in ks if e[7, k - 1] > 0])
+        out.append(f"  warpgroup {s}: {seg[0]} / {seg[1]} / {seg[2]} / {seg[3]}; "
+                   f"{end[0]} / {end[1]} / {nxt}")
     starts = tiles[5, 0][tiles[5, 0] > 0] - t0
     out.append(f"items {len(starts)}, starts (cycles from the CTA's first stamp) "
                f"{[int(x) for x in starts[:8]]}{' ...' if len(starts) > 8 else ''}; span "

@@ -248,6 +248,41 @@ def test_deterministic_bitwise():
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1], equal_nan=True)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("layout", ["BNSD", "TND"])
+def test_o_only_16_byte_aligned(layout, D):
+    """O rows leave the SM in 32-byte stores when O is 32-byte aligned and in
+    16-byte stores otherwise: an O that starts 16 bytes past a 32-byte
+    boundary gets the same bits, and the guard elements on both sides of it
+    stay untouched."""
+    if layout == "TND":
+        cu = [300, 700]
+        kw = _kw("TND", 2, 2, 700, 700, D, 3)
+        inp = random_inputs("TND", 2, 2, 700, 700, D, seed=93)
+        shape = (700, 2, D)
+        extra = dict(actual_seq_qlen=cu, actual_seq_kvlen=cu)
+    else:
+        kw = _kw("BNSD", 2, 2, 300, 333, D, 2)
+        inp = random_inputs("BNSD", 2, 2, 300, 333, D, seed=93)
+        shape = (2, 2, 300, D)
+        extra = {}
+    attn = fa.MaskedAttention(**kw)
+    q, k, v = (inp[x].cuda() for x in ("q", "k", "v"))
+    o_ref, l_ref = attn(q, k, v, **extra)
+    n = int(np.prod(shape))
+    raw = torch.full((n + 32,), -7.0, dtype=torch.bfloat16, device="cuda")
+    assert raw.data_ptr() % 256 == 0
+    o16 = raw[8:8 + n].view(shape)  # 16 bytes past a 256-byte boundary
+    l16 = torch.empty_like(l_ref)
+    attn(q, k, v, out=o16, lse=l16, **extra)
+    torch.cuda.synchronize()
+    attn.sync_status()
+    attn.close()
+    assert torch.equal(o16.view(torch.int16), o_ref.view(torch.int16))
+    assert torch.equal(l16.nan_to_num(0.0), l_ref.nan_to_num(0.0))
+    assert bool((raw[:8] == -7.0).all()) and bool((raw[8 + n:] == -7.0).all())
+
+
 def test_worked_split_examples_on_gpu():
     """Both cards of the sparseMode=7 and sparseMode=8 worked examples, each
     against the oracle, and their concatenation against the unsplit call."""
