@@ -969,13 +969,13 @@ __device__ __forceinline__ void exp_pack_part(const float (&x)[128], uint64_t m2
 }
 
 // ALiBi: scores of the row's 128 keys of this tile in log2 units with the
-// bias added, x <- x * scale_log2 + a2 * bias, a2 = slope * log2(e). d0 is
-// the signed distance of the tile's first key from the row's diagonal
-// anchored at the bottom-right corner (key c is d0 + c away). The linear
-// bias (right-aligned; the left-aligned one differs by a constant per row,
-// applied to lse at the end) is a ramp with one FMA per key; the square-root
-// variant takes sqrt of each distance's size on the MUFU unit and keeps its
-// sign. Hidden keys stay -inf.
+// bias added, a2 = slope * log2(e). d0 is the signed distance of the tile's
+// first key from the row's diagonal anchored at the bottom-right corner (key
+// c is d0 + c away). The linear bias (right-aligned; the left-aligned one
+// differs by a constant per row, applied to lse at the end) leaves
+// x <- x * scale_log2 + a2 * c, without the tile's offset a2 * d0; the
+// square-root variant adds its whole bias, x <- x * scale_log2 +
+// a2 * sign(d) sqrt|d|, with sqrt on the MUFU unit. Hidden keys stay -inf.
 __device__ __forceinline__ void apply_alibi(float (&x)[128], float scale_log2, float a2, int d0,
                                             bool sqrt_bias) {
   if (sqrt_bias) {
@@ -987,12 +987,23 @@ __device__ __forceinline__ void apply_alibi(float (&x)[128], float scale_log2, f
       x[c] = fmaf(x[c], scale_log2, a2 * copysignf(r, d));
     }
   } else {
-    const float base = a2 * (float)d0;
+    // The ramp a2 * c only: the tile's offset a2 * d0 is one scalar per row
+    // that the caller adds to the row maximum and to the exponent offset, so
+    // the ramp stays small and is built by additions (four interleaved chains
+    // of sixteen steps of 8 a2), one packed add per two keys.
     const uint64_t s2 = pack_f32x2(scale_log2, scale_log2);
+    const float st = 8.f * a2;
+    float r[8];
 #pragma unroll
-    for (int c = 0; c < 128; c += 2)
-      fma_x2(x[c], x[c + 1], s2,
-             pack_f32x2(fmaf((float)c, a2, base), fmaf((float)(c + 1), a2, base)));
+    for (int q = 0; q < 8; ++q) r[q] = a2 * (float)q;
+#pragma unroll
+    for (int c = 0; c < 128; c += 8) {
+#pragma unroll
+      for (int q = 0; q < 8; q += 2) {
+        fma_x2(x[c + q], x[c + q + 1], s2, pack_f32x2(r[q], r[q + 1]));
+        add_x2(r[q], r[q + 1], st, st);
+      }
+    }
   }
 }
 
@@ -1218,8 +1229,10 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
       // Without ALiBi the scale is applied inside the exponential (the max
       // of the raw scores scales, scale > 0); with it x holds the biased
       // scores in log2 units already.
+      // Linear ALiBi: the tile's bias offset, a2 * (distance of its first key).
+      const float abase = (kAlibi && p.alibi != 2) ? a2 * (float)(t * kTileN + dbase) : 0.f;
       if constexpr (kAlibi) apply_alibi(x, scale_log2, a2, t * kTileN + dbase, p.alibi == 2);
-      const float m_new = kAlibi ? row_max128(x) : row_max128(x) * scale_log2;
+      const float m_new = kAlibi ? row_max128(x) + abase : row_max128(x) * scale_log2;
       const bool resc = m_new > m_used + kRescaleLog2;
       float alpha = 1.f;
       if (resc) {
@@ -1239,7 +1252,8 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
       const float ref = ((m_used == -INFINITY) ? 0.f : m_used) + zero;
       const float mul = kAlibi ? 1.f : scale_log2;
       const uint64_t m2 = pack_f32x2(mul, mul);
-      const uint64_t c2 = pack_f32x2(-ref, -ref);
+      const float off = kAlibi ? abase - ref : -ref;
+      const uint64_t c2 = pack_f32x2(off, off);
       uint32_t pk[64];
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       // The other warpgroup gets its turn once the first kTokenCol keys are
