@@ -1060,6 +1060,32 @@ __device__ __forceinline__ void store_p_smem(uint32_t base, int row, const uint3
                  pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
 }
 
+// The same exponentials for all 128 keys, with P stored to shared memory as
+// it is produced: each 16-byte unit (8 keys) of row `row` of the P tile at
+// `base` (the layout of store_p_smem) is written as soon as it is
+// packed, so the stores overlap the exponential unit's work instead of
+// following it. Same sums as exp_pack_part.
+__device__ __forceinline__ void exp_pack_store(const float (&x)[128], uint64_t m2, uint64_t c2,
+                                               float (&acc)[8], uint32_t base, int row) {
+  const uint32_t rb = base + (uint32_t)row * 128u;
+  const uint32_t sw = (uint32_t)row & 7u;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float a = x[8 * u + 2 * q], b = x[8 * u + 2 * q + 1];
+      fma_x2(a, b, m2, c2);
+      a = ex2(a);
+      b = ex2(b);
+      add_x2(acc[2 * q], acc[2 * q + 1], a, b);
+      w[q] = pack_bf16(a, b);
+    }
+    st_shared_v4(rb + (uint32_t)(u >> 3) * 16384u + ((((uint32_t)u & 7u) ^ sw) << 4), w[0], w[1],
+                 w[2], w[3]);
+  }
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the
 // tensor core's (async-proxy) reads that follow the next barrier.
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -1243,49 +1269,17 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
       float zero = 0.f;
       if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 3, turn - 1);
       FA_WSTAMP(2, turn - 1);
-      if (!first_turn && !turn_wait(sub, m_new, zero, w.abort_flag)) {
-        ok = false;
-        break;
-      }
-      if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 4, turn - 1);
-      FA_WSTAMP(0, turn - 1);
-      const float ref = ((m_used == -INFINITY) ? 0.f : m_used) + zero;
-      const float mul = kAlibi ? 1.f : scale_log2;
-      const uint64_t m2 = pack_f32x2(mul, mul);
-      const float off = kAlibi ? abase - ref : -ref;
-      const uint64_t c2 = pack_f32x2(off, off);
-      uint32_t pk[64];
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      // The other warpgroup gets its turn once the first kTokenCol keys are
-      // done, so both feed the exponential unit across the handover.
-      // One instance of the exponential loop serves every tile while the
-      // FMA-pipe polynomial is off: a second copy for the (rarer) boundary
-      // tiles is cold in the instruction cache each time it runs.
-      if constexpr (kPolyPer8 > 0) {
-        if (partial) exp_pack_part<false, 0, kTokenCol>(x, m2, c2, acc, pk);
-        else exp_pack_part<true, 0, kTokenCol>(x, m2, c2, acc, pk);
-      } else {
-        exp_pack_part<false, 0, kTokenCol>(x, m2, c2, acc, pk);
-      }
-      __syncwarp();
-      turn_pass(sub ^ 1, ((acc[0] + acc[1]) + (acc[2] + acc[3])) +
-                             ((acc[4] + acc[5]) + (acc[6] + acc[7])));
-      if constexpr (kPolyPer8 > 0) {
-        if (partial) exp_pack_part<false, kTokenCol, 128>(x, m2, c2, acc, pk);
-        else exp_pack_part<true, kTokenCol, 128>(x, m2, c2, acc, pk);
-      } else {
-        exp_pack_part<false, kTokenCol, 128>(x, m2, c2, acc, pk);
-      }
-      l += sum_acc(acc);
-      if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 5, turn - 1);
-      FA_WSTAMP(1, turn - 1);
-      if (pv_count > 0) {
+      // With ALiBi the bias makes this warpgroup's work between two of its
+      // turns longer than the other warpgroup's exponentials, so P goes to
+      // shared memory while this turn's exponentials run (exp_pack_store),
+      // and the wait for the previous PV moves ahead of the turn. Without it
+      // that work fits, and stores inside the loop would only slow the
+      // exponentials: P is stored after the turn is handed over.
+      constexpr bool kStoreInTurn = kAlibi && !C::kPInTmem && kPolyPer8 == 0 && kTokenCol == 128;
+      auto pv_done = [&]() -> bool {
         // The previous PV of this sub-tile must be done: it still reads the
         // P buffer, and O_s must hold it before it is rescaled.
-        if (!wait_warp(&ctl->o_pv[sub], (pv_count - 1) & 1u, w, kSiteOPv)) {
-          ok = false;
-          break;
-        }
+        if (!wait_warp(&ctl->o_pv[sub], (pv_count - 1) & 1u, w, kSiteOPv)) return false;
         tc_fence_after();
         if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 6, turn - 1);
         // Not on the item's first tile: the first PV of an item overwrites O_s.
@@ -1299,13 +1293,71 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
             tmem_st32(tO + ch * 32u, ov);
           }
         }
+        return true;
+      };
+      if constexpr (kStoreInTurn) {
+        if (pv_count > 0 && !pv_done()) {
+          ok = false;
+          break;
+        }
       }
-      if constexpr (C::kPInTmem) {
-        tmem_st32(tP, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(tP + 32u, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
-      } else {
-        store_p_smem(sPs, row, pk);
+      if (!first_turn && !turn_wait(sub, m_new, zero, w.abort_flag)) {
+        ok = false;
+        break;
+      }
+      if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 4, turn - 1);
+      FA_WSTAMP(0, turn - 1);
+      const float ref = ((m_used == -INFINITY) ? 0.f : m_used) + zero;
+      const float mul = kAlibi ? 1.f : scale_log2;
+      const uint64_t m2 = pack_f32x2(mul, mul);
+      const float off = kAlibi ? abase - ref : -ref;
+      const uint64_t c2 = pack_f32x2(off, off);
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if constexpr (kStoreInTurn) {
+        exp_pack_store(x, m2, c2, acc, sPs, row);
+        __syncwarp();
+        turn_pass(sub ^ 1, ((acc[0] + acc[1]) + (acc[2] + acc[3])) +
+                               ((acc[4] + acc[5]) + (acc[6] + acc[7])));
+        l += sum_acc(acc);
         fence_proxy_async_smem();
+        if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 5, turn - 1);
+        FA_WSTAMP(1, turn - 1);
+      } else {
+        uint32_t pk[64];
+        // The other warpgroup gets its turn once the first kTokenCol keys
+        // are done, so both feed the exponential unit across the handover.
+        // One instance of the exponential loop serves every tile while the
+        // FMA-pipe polynomial is off: a second copy for the (rarer) boundary
+        // tiles is cold in the instruction cache each time it runs.
+        if constexpr (kPolyPer8 > 0) {
+          if (partial) exp_pack_part<false, 0, kTokenCol>(x, m2, c2, acc, pk);
+          else exp_pack_part<true, 0, kTokenCol>(x, m2, c2, acc, pk);
+        } else {
+          exp_pack_part<false, 0, kTokenCol>(x, m2, c2, acc, pk);
+        }
+        __syncwarp();
+        turn_pass(sub ^ 1, ((acc[0] + acc[1]) + (acc[2] + acc[3])) +
+                               ((acc[4] + acc[5]) + (acc[6] + acc[7])));
+        if constexpr (kPolyPer8 > 0) {
+          if (partial) exp_pack_part<false, kTokenCol, 128>(x, m2, c2, acc, pk);
+          else exp_pack_part<true, kTokenCol, 128>(x, m2, c2, acc, pk);
+        } else {
+          exp_pack_part<false, kTokenCol, 128>(x, m2, c2, acc, pk);
+        }
+        l += sum_acc(acc);
+        if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 5, turn - 1);
+        FA_WSTAMP(1, turn - 1);
+        if (pv_count > 0 && !pv_done()) {
+          ok = false;
+          break;
+        }
+        if constexpr (C::kPInTmem) {
+          tmem_st32(tP, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+          tmem_st32(tP + 32u, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+        } else {
+          store_p_smem(sPs, row, pk);
+          fence_proxy_async_smem();
+        }
       }
       tmem_st_wait();
       tc_fence_before();
