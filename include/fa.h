@@ -419,7 +419,7 @@ fa_status_t fa_plan_stats(const fa_desc_t* desc, const int64_t* prefix,
  * shorter's). A list each CTA takes a fixed share of (fewer than 8 items
  * per SM) is longest first, ties in (sequence, block, head) order. A list
  * that is claimed at run time (at least 8 items per SM) is longest first by
- * buckets of 16 key tiles (key / 128), and inside a bucket ordered by
+ * buckets of 24 key tiles (key / 192), and inside a bucket ordered by
  * (sequence, head), then longest first, then block: the items in flight
  * then share their K/V tiles through L2. Items without a key tile come last
  * in both orders. Item m is out[4m .. 4m+3] = (sequence b, head h, block of

@@ -485,8 +485,8 @@ def _expected_keys(c, prefix, cu_q, cu_kv):
 @pytest.mark.parametrize("num_sms", [148, 8])
 def test_claimed_list_order_groups_sequence_and_head_inside_length_buckets(num_sms):
     """A list with at least 8 items per SM (claimed at run time) is ordered for
-    L2 locality: items without a key tile last, then buckets of 16 key tiles
-    (key // 128) longest first, inside a bucket (sequence, head) ascending,
+    L2 locality: items without a key tile last, then buckets of 24 key tiles
+    (key // 192) longest first, inside a bucket (sequence, head) ascending,
     then the key descending, then the block; every item once with the oracle's
     key. With fewer items per SM the same call gives the strict order."""
     g = np.random.default_rng(9)
@@ -509,7 +509,7 @@ def test_claimed_list_order_groups_sequence_and_head_inside_length_buckets(num_s
     assert zero.any() and not np.any(zero[:-1] & ~zero[1:]), "items without a key tile last"
     k = keys[~zero]
     it = items[~zero]
-    buckets = k // 128
+    buckets = k // 192
     assert np.all(buckets[:-1] >= buckets[1:])
     for m in range(len(it) - 1):
         if buckets[m] == buckets[m + 1]:
