@@ -496,6 +496,22 @@ __device__ __forceinline__ int item_index(int k) {
   return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
 
+// Walk over an item's key tiles [lo, hi): ascending, or, with kRev (the
+// ALiBi instances), descending from the diagonal. ALiBi raises a row's
+// scores towards the diagonal by up to slope * 128 per tile, so an
+// ascending walk raises the running maximum on almost every tile, and every
+// raise by more than the rescale threshold rescales O; walking down from the
+// diagonal meets the largest bias first. Written so that the ascending walk
+// compiles to the plain loop.
+template <bool kRev>
+__device__ __forceinline__ int walk_first(int lo, int hi) { return kRev ? hi - 1 : lo; }
+template <bool kRev>
+__device__ __forceinline__ bool walk_in(int t, int lo, int hi) { return kRev ? t >= lo : t < hi; }
+template <bool kRev>
+__device__ __forceinline__ int walk_last(int lo, int hi) { return kRev ? lo : hi - 1; }
+template <bool kRev>
+constexpr int kWalkStep = kRev ? -1 : 1;
+
 struct ItemPlan {
   TileRange tr[2];
   int lo, hi;      // union of the two sub-tiles' tile ranges
@@ -557,7 +573,7 @@ __device__ __forceinline__ bool active(const TileRange& t, int j) { return j >= 
 // With kClaim this thread also takes the CTA's items: it publishes the index
 // of each into the ring, the next one once its claim returns, before the
 // loads the other roles need to finish the current item.
-template <int D, bool kOcc, bool kClaim>
+template <int D, bool kOcc, bool kClaim, bool kRev>
 __device__ void load_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint8_t* sQ,
                           uint8_t* sKV, const WaitCtx& w) {
   using C = Cfg<D>;
@@ -607,17 +623,19 @@ __device__ void load_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint8_t
     const ItemPlan ip = plan_item<kOcc>(p, idx, it, sr);
     if (ip.hi <= ip.lo) continue;
     const int bc = p.tnd ? 0 : it.b;
+    constexpr int st = kWalkStep<kRev>;
     if (ip.tr[0].hi > ip.tr[0].lo) ok = load_q(it, sr, 0, bc);
-    if (ok) ok = load_kv(&p.tm_k, sr.kv_off + ip.lo * kTileN, it.h, bc);
+    if (ok) ok = load_kv(&p.tm_k, sr.kv_off + walk_first<kRev>(ip.lo, ip.hi) * kTileN, it.h, bc);
     if (ok && ip.tr[1].hi > ip.tr[1].lo) ok = load_q(it, sr, 1, bc);
     // The previous item's last V follows this item's first K: the MMA warp
     // computes those scores before it finishes the previous item.
     if (ok && pend.h >= 0) ok = load_kv(&p.tm_v, pend.row, pend.h, pend.bc);
-    for (int t = ip.lo; t + 1 < ip.hi && ok; ++t) {
-      ok = load_kv(&p.tm_k, sr.kv_off + (t + 1) * kTileN, it.h, bc);
+    for (int t = walk_first<kRev>(ip.lo, ip.hi); walk_in<kRev>(t + st, ip.lo, ip.hi) && ok;
+         t += st) {
+      ok = load_kv(&p.tm_k, sr.kv_off + (t + st) * kTileN, it.h, bc);
       if (ok) ok = load_kv(&p.tm_v, sr.kv_off + t * kTileN, it.h, bc);
     }
-    pend = PendingV{sr.kv_off + (ip.hi - 1) * kTileN, it.h, bc};
+    pend = PendingV{sr.kv_off + walk_last<kRev>(ip.lo, ip.hi) * kTileN, it.h, bc};
   }
   } else {
   int idx = item_index(0);
@@ -638,22 +656,26 @@ __device__ void load_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint8_t
     bool claimed = false;
     if (ok && ip.hi > ip.lo) {
       const int bc = p.tnd ? 0 : it.b;
-      const int claim_at = max(ip.lo, ip.hi - 1 - kClaimLead);
+      constexpr int st = kWalkStep<kRev>;
+      // kClaimLead tiles before the walk's last
+      const int claim_at = kRev ? min(ip.hi - 1, ip.lo + kClaimLead)
+                                : max(ip.lo, ip.hi - 1 - kClaimLead);
       if (ip.tr[0].hi > ip.tr[0].lo) ok = load_q(it, sr, 0, bc);
-      if (ok) ok = load_kv(&p.tm_k, sr.kv_off + ip.lo * kTileN, it.h, bc);
+      if (ok) ok = load_kv(&p.tm_k, sr.kv_off + walk_first<kRev>(ip.lo, ip.hi) * kTileN, it.h, bc);
       if (ok && ip.tr[1].hi > ip.tr[1].lo) ok = load_q(it, sr, 1, bc);
       if (ok && pend.h >= 0) ok = load_kv(&p.tm_v, pend.row, pend.h, pend.bc);
-      for (int t = ip.lo; t + 1 < ip.hi && ok; ++t) {
+      for (int t = walk_first<kRev>(ip.lo, ip.hi); walk_in<kRev>(t + st, ip.lo, ip.hi) && ok;
+           t += st) {
         // The claim's result is first used after this loop, so its round
         // trip overlaps the item's last loads.
-        if (!claimed && t >= claim_at) {
+        if (!claimed && (kRev ? t <= claim_at : t >= claim_at)) {
           ticket = atomicAdd(p.claim, 1u);
           claimed = true;
         }
-        ok = load_kv(&p.tm_k, sr.kv_off + (t + 1) * kTileN, it.h, bc);
+        ok = load_kv(&p.tm_k, sr.kv_off + (t + st) * kTileN, it.h, bc);
         if (ok) ok = load_kv(&p.tm_v, sr.kv_off + t * kTileN, it.h, bc);
       }
-      pend = PendingV{sr.kv_off + (ip.hi - 1) * kTileN, it.h, bc};
+      pend = PendingV{sr.kv_off + walk_last<kRev>(ip.lo, ip.hi) * kTileN, it.h, bc};
     }
     if (!ok) break;
     if (!claimed) ticket = atomicAdd(p.claim, 1u);
@@ -783,7 +805,7 @@ __device__ __forceinline__ uint32_t ring_v(uint32_t g, bool last) {
 // It runs ahead of the P.V stream (another thread), limited only by the
 // softmax releasing S, so the scores of the next tile, also across item
 // boundaries, are ready when the softmax wants them.
-template <int D, bool kOcc, bool kClaim>
+template <int D, bool kOcc, bool kClaim, bool kRev>
 __device__ void qk_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t tmem,
                         const uint8_t* sQ, const uint8_t* sKV, const WaitCtx& w) {
   using C = Cfg<D>;
@@ -796,7 +818,8 @@ __device__ void qk_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
   MmaPlan cur;
   while (ok && next_item<kOcc, kClaim>(p, ctl, w, k, cur)) {
     bool q_ready[2] = {false, false};
-    for (int t = cur.lo[2]; t < cur.hi[2] && ok; ++t, ++g) {
+    for (int t = walk_first<kRev>(cur.lo[2], cur.hi[2]); walk_in<kRev>(t, cur.lo[2], cur.hi[2]) && ok;
+         t += kWalkStep<kRev>, ++g) {
       const uint32_t r = ring_k(g);
       FA_STAMP(2, 0, g);
       if (!wait_bounded(&ctl->kv_full[r % NS], (r / NS) & 1u, w, kSiteKvFull)) {
@@ -825,7 +848,8 @@ __device__ void qk_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
         issue_qk<D>(tmem, sQ, sKV, s, r % NS);
         mma_commit(&ctl->s_full[s]);
         ++n_qk[s];
-        if (t == cur.hi[s] - 1) mma_commit(&ctl->q_empty[s]);  // last read of this Q
+        // last read of this Q
+        if (t == walk_last<kRev>(cur.lo[s], cur.hi[s])) mma_commit(&ctl->q_empty[s]);
       }
       if (ok) mma_commit(&ctl->kv_empty[r % NS]);
     }
@@ -841,7 +865,7 @@ __device__ void qk_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
 // the commit after it tells the softmax that O_s is updated and that the P
 // buffer may be rewritten. The first PV of an item overwrites O_s, so it
 // waits until the epilogue has read O_s of the previous item that had one.
-template <int D, bool kOcc, bool kClaim>
+template <int D, bool kOcc, bool kClaim, bool kRev>
 __device__ void pv_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t tmem,
                         const uint8_t* sP, const uint8_t* sKV, const WaitCtx& w) {
   using C = Cfg<D>;
@@ -859,8 +883,9 @@ __device__ void pv_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, uint32_t 
     bool have_next = false;
     if constexpr (!kClaim) have_next = next_item<kOcc, false>(p, ctl, w, k, nxt);
     bool first[2] = {true, true};
-    for (int t = cur.lo[2]; t < cur.hi[2] && ok; ++t, ++g) {
-      const bool last_t = t + 1 == cur.hi[2];
+    for (int t = walk_first<kRev>(cur.lo[2], cur.hi[2]); walk_in<kRev>(t, cur.lo[2], cur.hi[2]) && ok;
+         t += kWalkStep<kRev>, ++g) {
+      const bool last_t = t == walk_last<kRev>(cur.lo[2], cur.hi[2]);
       if constexpr (kClaim) {
         // A claimed next item is known once the TMA thread's claim returns,
         // published before it loads this item's last V: look at one slot at
@@ -1182,9 +1207,11 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
           asm volatile("prefetch.global.L1 [%0];" ::"l"(mrow + (int64_t)tn * kTileN));
       }
     };
-    prefetch_mask(tr.lo);
+    prefetch_mask(walk_first<kAlibi>(tr.lo, tr.hi));
     if (stamper) FA_STAMP_DEP(sub ? 7 : 5, 4, k, jlo ^ jhi);
-    for (int t = ip.lo; t < ip.hi; ++t) {
+    // The ALiBi instances walk the tiles down from the diagonal (walk_first).
+    for (int t = walk_first<kAlibi>(ip.lo, ip.hi); walk_in<kAlibi>(t, ip.lo, ip.hi);
+         t += kWalkStep<kAlibi>) {
       // Turn on the exponential unit: warpgroup 0 goes first in every tile.
       const bool first_turn = sub == 0 && turn == 0;
       ++turn;
@@ -1198,7 +1225,7 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
         turn_pass(sub ^ 1, zero);
         continue;
       }
-      prefetch_mask(t + 1);
+      prefetch_mask(t + kWalkStep<kAlibi>);
       if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 0, turn - 1);
       if (!wait_warp(&ctl->s_full[sub], s_count & 1u, w, kSiteSFull)) {
         ok = false;
@@ -1282,8 +1309,9 @@ __device__ void softmax_role(const FwdParams& p, Ctl<Cfg<D>::kStages>* ctl, floa
         if (!wait_warp(&ctl->o_pv[sub], (pv_count - 1) & 1u, w, kSiteOPv)) return false;
         tc_fence_after();
         if ((threadIdx.x & 127) == 0) FA_STAMP(sub, 6, turn - 1);
-        // Not on the item's first tile: the first PV of an item overwrites O_s.
-        if (t > tr.lo && __any_sync(0xffffffffu, resc)) {
+        // Not on the sub-tile's first tile of the item: the first PV of an
+        // item overwrites O_s.
+        if ((kAlibi ? t < tr.hi - 1 : t > tr.lo) && __any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
           for (int ch = 0; ch < D / 32; ++ch) {
             uint32_t ov[32];
@@ -1532,9 +1560,9 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100(const __grid_constan
     epilogue_role<D, kOcc, kClaim>(p, ctl, inv_l_sm, tmem, w);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
-    if (warp == kWarpMma && lane == 0) qk_role<D, kOcc, kClaim>(p, ctl, tmem, sQ, sKV, w);
-    if (warp == kWarpPv && lane == 0) pv_role<D, kOcc, kClaim>(p, ctl, tmem, sP, sKV, w);
-    if (warp == kWarpLoad && lane == 0) load_role<D, kOcc, kClaim>(p, ctl, sQ, sKV, w);
+    if (warp == kWarpMma && lane == 0) qk_role<D, kOcc, kClaim, kAlibi>(p, ctl, tmem, sQ, sKV, w);
+    if (warp == kWarpPv && lane == 0) pv_role<D, kOcc, kClaim, kAlibi>(p, ctl, tmem, sP, sKV, w);
+    if (warp == kWarpLoad && lane == 0) load_role<D, kOcc, kClaim, kAlibi>(p, ctl, sQ, sKV, w);
   }
   __syncwarp();
   tc_fence_before();

@@ -106,14 +106,24 @@ def summarize(tiles, warps) -> str:
     """The tables described in the module docstring, as text."""
     out = []
     t0 = tiles[tiles > 0].min()
-    phases = ["S wait", "S load+mask", "row max", "turn wait", "exponentials", "PV wait",
-              "P store"]
-    out.append("| warpgroup | tiles | " + " | ".join(phases) + " | turn period |")
-    out.append("|---" * (len(phases) + 3) + "|")
+    names = {1: "S wait", 2: "S load+mask", 3: "row max", 4: "turn wait", 5: "exponentials",
+             6: "PV wait", 7: "P store"}
+    # Events in the order they occur: 0 S wait, 1 S ready, 2 S loaded, 3 row
+    # maximum, then either 4 turn, 5 exponentials done, 6 previous PV done,
+    # 7 P handed over, or (P stored inside the exponential loop) 6 before 4.
+    e0 = tiles[0]
+    both = np.nonzero((e0[4] > 0) & (e0[6] > 0))[0]
+    pv_first = len(both) > 0 and np.median(e0[6, both] - e0[4, both]) < 0
+    order = [0, 1, 2, 3, 6, 4, 5, 7] if pv_first else list(range(8))
+    if pv_first:
+        names.update({6: "PV wait", 4: "turn wait", 5: "exponentials + P store", 7: "P hand-over"})
+    out.append("| warpgroup | tiles | " + " | ".join(names[k] for k in order[1:]) +
+               " | turn period |")
+    out.append("|---" * (len(order) + 2) + "|")
     for s in (0, 1):
         e = tiles[s]
         idx = np.nonzero((e[0] > 0) & (e[7] > 0))[0]
-        d = np.diff(e[:, idx], axis=0)
+        d = np.diff(e[order][:, idx], axis=0)
         per = np.diff(e[4, idx])
         out.append(f"| {s} | {len(idx)} | " + " | ".join(str(_med(d[i])) for i in range(7))
                    + f" | {_med(per)} |")
