@@ -44,9 +44,9 @@ bool claims_items(int64_t n_items, int num_sms);
 // from as many (sequence, head) pairs, whose K/V outgrow L2 and are read
 // from DRAM by every item: 3.7x the algorithmic bytes on a causal-prefix
 // problem of 8k tokens, 4.5x on 16 varlen sequences). Items without a key
-// tile come last either way (claiming relies on it). Buckets of 24 tiles
-// measured 1-1.3 % faster than 16 on both (8: 2.5-4 % slower; 64: varlen
-// +3 %, prefix -2 %).
+// tile come last either way (claiming relies on it). On those two problems
+// buckets of 24 tiles measured 1-1.3 % faster than 16 (8: 2.5-4 % slower;
+// 64: the 16 sequences +3 %, the 8k-token problem -2 %).
 constexpr int32_t kLocalityTiles = 24;
 void order_work_list(WorkItem* first, WorkItem* last, bool locality);
 int64_t visible_pairs(const fa_desc_t* d, const std::vector<SeqRec>& recs);
