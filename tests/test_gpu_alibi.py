@@ -94,6 +94,43 @@ def test_alibi_on_claimed_work_is_deterministic():
     assert_close(a[0], a[1], o_ref, lse_ref, "claimed ALiBi")
 
 
+@pytest.mark.parametrize("kind", ["right", "left", "sqrt"])
+def test_alibi_claimed_long_items_sampled_rows(kind):
+    """Claimed ALiBi work whose items span up to 9 key tiles, so that the
+    claim, the Q releases and the last V of the descending walk fall in the
+    middle of long items: 260 varlen sequences of 500-1100 query rows x 4
+    heads (about 3,700 items), slopes from steep to flat; 600 sampled rows
+    against the oracle row by row, and the same bits on a second call."""
+    g = torch.Generator().manual_seed(3200)
+    nseq = 260
+    sq = torch.randint(500, 1101, (nseq,), generator=g)
+    skv = sq + torch.randint(0, 100, (nseq,), generator=g)
+    cu_q, cu_kv = torch.cumsum(sq, 0).tolist(), torch.cumsum(skv, 0).tolist()
+    N, D = 4, 128
+    kw = dict(layout="TND", B=nseq, N=N, Sq=cu_q[-1], Skv=cu_kv[-1], D=D, sparse_mode=3,
+              alibi=kind)
+    items = fa.fa_plan_stats(fa.make_desc(**kw), actual_seq_qlen=cu_q, actual_seq_kvlen=cu_kv)[0]
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert items >= fa.CLAIM_MIN_ITEMS_PER_CTA * sms
+    inp = random_inputs("TND", nseq, N, cu_q[-1], cu_kv[-1], D, seed=3201)
+    slopes = [0.71, 0.125, 0.02, 0.0039]
+    a = _run(kw, inp, slopes, None, cu_q, cu_kv)
+    b = _run(kw, inp, slopes, None, cu_q, cu_kv)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    pkw = {k_: v_ for k_, v_ in kw.items() if k_ != "alibi"}
+    pb = problem_of(pkw, None, None, cu_q, cu_kv)
+    gr = np.random.default_rng(3202)
+    q_off = [0] + cu_q[:-1]
+    rows = []  # (sequence, head, row inside the sequence)
+    for b, h in zip(gr.integers(0, nseq, 600), gr.integers(0, N, 600)):
+        rows.append((int(b), int(h), int(gr.integers(0, int(sq[b])))))
+    o_ref, l_ref = oracle.attention_rows(pb, inp["q"], inp["k"], inp["v"], rows, alibi=kind,
+                                         slopes=slopes)
+    o_got = np.stack([a[0][q_off[b] + i, h] for b, h, i in rows])
+    l_got = np.array([a[1][h, q_off[b] + i] for b, h, i in rows])
+    assert_close(o_got, l_got, o_ref, l_ref, f"claimed ALiBi ({kind}), long items")
+
+
 def test_alibi_left_equals_right_in_o():
     """Left- and right-aligned biases give the same weights: equal O bits up
     to the last rounding (the kernel computes both through the same
