@@ -529,3 +529,51 @@ def test_trace_build_compiles_and_exports_its_accessors():
     assert lib.fa_trace_cta() == 3
     prod = fa.load_library()
     assert not hasattr(prod, "fa_trace_read")
+
+
+def _synthetic_trace(pv_first):
+    """Stamp arrays of two warpgroups over 20 turns with fixed phase lengths:
+    S wait 100, load 50, max 200, then turn wait 300, exponentials 1000, PV
+    wait 80, P store 400 (or, pv_first, PV wait 80 before the turn wait)."""
+    import numpy as np
+    tiles = np.zeros((8, 8, 1024), dtype=np.int64)
+    warps = np.zeros((8, 4, 1024), dtype=np.int64)
+    for s in (0, 1):
+        t = 1000 + 500 * s
+        for i in range(20):
+            ev = {0: t, 1: t + 100, 2: t + 150, 3: t + 350}
+            if pv_first:
+                ev.update({6: t + 430, 4: t + 730, 5: t + 1730, 7: t + 1790})
+            else:
+                ev.update({4: t + 650, 5: t + 1650, 6: t + 1730, 7: t + 2130})
+            for e, v in ev.items():
+                tiles[s, e, i] = v
+            for wq in range(4):
+                warps[4 * s + wq, 0, i] = ev[4]
+                warps[4 * s + wq, 1, i] = ev[5]
+            t += 3000
+    return tiles, warps
+
+
+@pytest.mark.parametrize("pv_first", [False, True])
+def test_trace_summary_phases_follow_the_event_order(pv_first):
+    """The trace tool's table lists each turn's phases in the order they
+    occur: with the previous PV awaited before the turn (the ALiBi instances)
+    its columns follow that order, and every phase length is recovered."""
+    from masked_attention_fa_b200.trace import summarize
+    tiles, warps = _synthetic_trace(pv_first)
+    lines = summarize(tiles, warps).splitlines()
+    head = [c.strip() for c in lines[0].strip("|").split("|")]
+    row0 = [c.strip() for c in lines[2].strip("|").split("|")]
+    got = dict(zip(head[2:-1], (int(v) for v in row0[2:-1])))
+    if pv_first:
+        assert list(got) == ["S wait", "S load+mask", "row max", "PV wait", "turn wait",
+                             "exponentials + P store", "P hand-over"]
+        assert got == {"S wait": 100, "S load+mask": 50, "row max": 200, "PV wait": 80,
+                       "turn wait": 300, "exponentials + P store": 1000, "P hand-over": 60}
+    else:
+        assert list(got) == ["S wait", "S load+mask", "row max", "turn wait", "exponentials",
+                             "PV wait", "P store"]
+        assert got == {"S wait": 100, "S load+mask": 50, "row max": 200, "turn wait": 300,
+                       "exponentials": 1000, "PV wait": 80, "P store": 400}
+    assert int(row0[-1]) == 3000  # turn period
