@@ -75,6 +75,8 @@ def record(workload: str, cta: int):
     inp = make_inputs(w)
     q, k, v = (inp[x].cuda() for x in ("q", "k", "v"))
     arrays = bench.workload_args(w)
+    if inp["mask"] is not None:
+        arrays["atten_mask"] = inp["mask"].cuda()
     attn = fa.MaskedAttention(w.layout, w.B, w.N, w.Sq, w.Skv, w.D, w.sparse_mode, w.pre_tokens,
                               w.next_tokens, w.scale, w.mask_kind, w.alibi)
     slopes = torch.tensor(alibi_slopes(w.N), device="cuda") if w.alibi else None
